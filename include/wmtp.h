@@ -1,0 +1,245 @@
+/*
+ * wmtp.h -- C ABI of libwmtp: the per-decode-step attention of Windowed-MTP
+ * speculative decoding on one NVIDIA B200 (sm_100a).
+ *
+ * The method (from "Windowed-MTP: Removing the Full-Context Draft-KV Tax at
+ * Million-Token Context", arxivlens paper view, Abstract): a built-in MTP
+ * draft head runs gamma single-token decode attentions per decode step.  Run
+ * natively, each one reads the draft layer's whole KV cache; Windowed-MTP
+ * restricts the draft (only the draft) to S attention-sink tokens plus a
+ * sliding window of the last W tokens, kept in a compact ring buffer.  The
+ * target then verifies gamma+1 tokens with causal attention over its full
+ * paged KV, so accepted tokens are unchanged.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument that is not a params/ring/kv descriptor is DEVICE
+ *   memory owned by the caller.  Descriptor structs themselves are read on the
+ *   host during the call and may be freed when it returns.  The library never
+ *   allocates device memory.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream) and never synchronise the host.
+ * - Host-detectable argument errors return a negative wmtp_status before
+ *   anything is launched.
+ * - Device-detected problems (a page-table entry outside the pool, a length
+ *   out of range, an inconsistent ring state) are OR-ed as WMTP_DEV_* bits
+ *   into *status_word when status_word is non-NULL; the offending tile or
+ *   sequence is skipped.  No kernel traps; every wait inside a kernel is
+ *   bounded and reports WMTP_DEV_TIMEOUT if it gives up.
+ * - bf16 means IEEE bfloat16 (raw 16-bit storage); fp32 accumulation.
+ * - Supported shapes: head_dim in {64, 256}; num_heads_q / num_heads_kv = G
+ *   with rows = num_q * G in 1..64 (rows are padded to a multiple of 8);
+ *   page_size in {16, 32, 64, 128, 256}; gamma_max <= 16.  Anything else
+ *   returns WMTP_ERR_UNSUPPORTED.
+ *
+ * Layouts
+ * -------
+ *   paged K or V pool : [num_pages][Hkv][page_size][D]      bf16
+ *   page_table        : [batch][max_pages]                  int32
+ *   kv_len            : [batch]                             int32
+ *   draft query       : [batch][Hq][D]                      bf16
+ *   verify query      : [batch][num_q][Hq][D]               bf16
+ *   ring K or V       : [batch][Hkv][S+W][D]                bf16
+ *   ring tags         : [batch][S+W]                        int32 (-1 = empty)
+ *   undo K or V       : [batch][gamma_max][Hkv][D]          bf16
+ *   output            : like the query, fp32 or bf16 (out_fp32)
+ *   lse_out           : [batch][num_q][Hq] fp32, natural log (NULL = skip)
+ *
+ * Query head h reads KV head h / G (G = Hq / Hkv).
+ */
+#ifndef WMTP_H_
+#define WMTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WMTP_OK = 0,
+  WMTP_ERR_INVALID_ARG = -1, /* NULL where a pointer is required, bad size */
+  WMTP_ERR_UNSUPPORTED = -2, /* a shape outside the supported set */
+  WMTP_ERR_WORKSPACE = -3,   /* workspace too small or misaligned */
+  WMTP_ERR_CUDA = -4         /* a CUDA runtime call failed (launch, attribute) */
+} wmtp_status;
+
+/* Bits the kernels OR into *status_word. */
+#define WMTP_DEV_PAGE_OOB 0x1   /* page-table entry outside [0, num_pages) */
+#define WMTP_DEV_LEN_OOB 0x2    /* kv_len < num_q or > max_pages * page_size */
+#define WMTP_DEV_RING_STATE 0x4 /* ring len/committed inconsistent, or
+                                   truncate_to outside [committed, len] */
+#define WMTP_DEV_UNDO_FULL 0x8  /* speculative appends beyond gamma_max */
+#define WMTP_DEV_TIMEOUT 0x10   /* a bounded in-kernel wait gave up */
+
+typedef struct {
+  int32_t num_heads_q;  /* Hq */
+  int32_t num_heads_kv; /* Hkv; Hq % Hkv == 0 */
+  int32_t head_dim;     /* D */
+  int32_t page_size;    /* P, tokens per page of the paged pools */
+  int32_t sinks;        /* S, attention-sink tokens of the windowed draft */
+  int32_t window;       /* W, sliding-window tokens of the windowed draft (>= 1) */
+  int32_t gamma_max;    /* undo-log capacity: speculative appends per commit */
+  float sm_scale;       /* softmax scale; 0 means 1/sqrt(D) */
+} wmtp_params;
+
+/* One attention layer's paged KV cache (all device pointers). */
+typedef struct {
+  void* k_pool;              /* [num_pages][Hkv][P][D] bf16 */
+  void* v_pool;              /* [num_pages][Hkv][P][D] bf16 */
+  int32_t num_pages;
+  const int32_t* page_table; /* [batch][max_pages] */
+  int32_t max_pages;
+  const int32_t* kv_len;     /* [batch] valid tokens per sequence */
+} wmtp_paged_kv;
+
+/* Per-sequence compact draft ring buffers (all device pointers).  The ring
+ * holds positions {0..min(S,len)-1} U {max(S,len-W)..len-1}; position p lives
+ * in slot p if p < S, else S + (p - S) mod W. */
+typedef struct {
+  void* k;             /* [batch][Hkv][S+W][D] bf16 */
+  void* v;             /* [batch][Hkv][S+W][D] bf16 */
+  int32_t* tags;       /* [batch][S+W] position held by each slot, -1 = empty */
+  int32_t* len;        /* [batch] positions appended (speculative included) */
+  int32_t* committed;  /* [batch] length at the last commit */
+  void* undo_k;        /* [batch][gamma_max][Hkv][D] bf16, overwritten entries */
+  void* undo_v;        /* [batch][gamma_max][Hkv][D] bf16 */
+  int32_t* undo_tags;  /* [batch][gamma_max] tags of the overwritten entries */
+  int32_t batch;
+} wmtp_ring;
+
+/* Status as a static string ("ok", "invalid argument", ...). */
+const char* wmtp_status_string(int32_t status);
+
+/* Library version as "major.minor.patch". */
+const char* wmtp_version(void);
+
+/*
+ * wmtp_draft_attn_full -- native MTP draft attention.
+ * Source: arxivlens view of the paper, Abstract (the draft head attends over
+ * the full KV cache in each of its gamma forwards); howtospark case study
+ * "Does speculative decode still pay at 128K context?", Background.
+ *
+ * For every sequence b and query head h: o = softmax(sm_scale * K q) V over
+ * positions 0 .. kv_len[b]-1 of the draft layer's paged cache (kv_len
+ * includes the token appended for this draft step).
+ *   q        : [batch][Hq][D] bf16
+ *   kv       : the draft layer's paged cache
+ *   out      : [batch][Hq][D], fp32 if out_fp32 else bf16
+ *   lse_out  : [batch][Hq] fp32 or NULL.
+ *   kv_len[b] == 0 is an empty sequence: o = 0, lse = -inf.  A kv_len below
+ *   num_q or above max_pages * page_size sets WMTP_DEV_LEN_OOB and is treated
+ *   as empty.
+ *   workspace: device scratch for split-KV partials, 256-byte aligned.  Call
+ *              with workspace == NULL to get the size in *workspace_bytes
+ *              (nothing is launched).  The size depends on the device's SM
+ *              count, batch, shapes and max_pages.
+ */
+wmtp_status wmtp_draft_attn_full(const wmtp_params* params, int32_t batch, const void* q,
+                                 const wmtp_paged_kv* kv, void* out, int32_t out_fp32,
+                                 float* lse_out, void* workspace, size_t* workspace_bytes,
+                                 int32_t* status_word, void* stream);
+
+/*
+ * wmtp_draft_attn_windowed -- Windowed-MTP draft attention over the ring.
+ * Source: arxivlens view, Abstract (StreamingLLM-style sink plus window on the
+ * draft only; the compact ring buffer); readpriors post "Your Million-Token
+ * Pipeline Is Bleeding Speed ...", What happened.
+ *
+ * For every sequence b and head h: o = softmax(sm_scale * K q) V over the ring
+ * entries whose tag t satisfies t < min(S, len[b]) or
+ * max(S, len[b] - W) <= t < len[b].  Reads at most S+W entries per sequence,
+ * whatever the context length.
+ *   q: [ring->batch][Hq][D] bf16; out / lse_out / workspace as above.
+ */
+wmtp_status wmtp_draft_attn_windowed(const wmtp_params* params, const void* q,
+                                     const wmtp_ring* ring, void* out, int32_t out_fp32,
+                                     float* lse_out, void* workspace, size_t* workspace_bytes,
+                                     int32_t* status_word, void* stream);
+
+/*
+ * wmtp_ring_append -- append draft K/V to the rings, with speculative undo.
+ * Source: arxivlens view, Abstract and Technical contributions (a compact
+ * ring buffer holding only the sink and window entries).  The undo log is
+ * this library's reading of how a speculative draft token that the target
+ * rejects is taken back out of the ring (the pages do not say).
+ *
+ * Per sequence b, in order:
+ *   1. if truncate_to != NULL and truncate_to[b] >= 0: roll back to length
+ *      truncate_to[b] (must lie in [committed[b], len[b]]), restoring the
+ *      entries the rolled-back speculative appends overwrote, newest first;
+ *   2. append n_new[b] tokens (k_new/v_new rows 0..n_new[b]-1) at positions
+ *      len[b] .. len[b]+n_new[b]-1.  If speculative, each append first saves
+ *      the entry it overwrites to the undo log (at most gamma_max since the
+ *      last commit); otherwise only the tokens that survive in the final
+ *      sink + window are written;
+ *   3. if !speculative: commit (committed[b] = len[b]; undo log emptied).
+ *   k_new, v_new: [batch][max_new][Hkv][D] bf16; n_new: [batch], each in
+ *   [0, max_new]; n_new may be NULL when max_new == 0.
+ * Results are bit-exact copies of the given bf16 values.
+ */
+wmtp_status wmtp_ring_append(const wmtp_params* params, const wmtp_ring* ring,
+                             const int32_t* truncate_to, const int32_t* n_new,
+                             const void* k_new, const void* v_new, int32_t max_new,
+                             int32_t speculative, int32_t* status_word, void* stream);
+
+/*
+ * wmtp_ring_reset -- empty every ring: tags = -1, K/V and undo zeroed,
+ * len = committed = 0.  Call once before first use.
+ */
+wmtp_status wmtp_ring_reset(const wmtp_params* params, const wmtp_ring* ring, void* stream);
+
+/*
+ * wmtp_verify_attn -- target verify attention of num_q = gamma+1 queries.
+ * Source: arxivlens view, Abstract (verification keeps full-context attention,
+ * so the target distribution is preserved); howtospark case study, Method (one
+ * cycle = gamma draft forwards plus one batched verify).
+ *
+ * Query i (0 <= i < num_q) of sequence b sits at position kv_len[b]-num_q+i
+ * and attends causally to positions 0 .. kv_len[b]-num_q+i of the layer's
+ * paged cache; the caller has already written the num_q new tokens' K/V.
+ * All G query heads of a KV head and all num_q queries are processed together
+ * so each K/V byte is read once.
+ *   q: [batch][num_q][Hq][D] bf16; out: [batch][num_q][Hq][D];
+ *   lse_out: [batch][num_q][Hq]; workspace as for wmtp_draft_attn_full.
+ */
+wmtp_status wmtp_verify_attn(const wmtp_params* params, int32_t batch, int32_t num_q,
+                             const void* q, const wmtp_paged_kv* kv, void* out,
+                             int32_t out_fp32, float* lse_out, void* workspace,
+                             size_t* workspace_bytes, int32_t* status_word, void* stream);
+
+/*
+ * wmtp_splitkv_combine -- merge split-KV partial attention results.
+ * Not on the pages: the standard log-sum-exp identity behind split-KV
+ * (flash-decoding) decode attention, needed to spread one sequence over the
+ * GPU's SMs.  For each row r:
+ *   m = max_s lse[r][s];  w_s = exp(lse[r][s] - m);
+ *   out[r] = sum_s w_s part_o[r][s] / sum_s w_s;  lse_out[r] = m + log sum_s w_s.
+ * Splits with lse = -inf carry no weight; a row whose splits are all empty
+ * gives out = 0, lse = -inf.
+ *   part_o: [rows][nsplit][head_dim] fp32; part_lse: [rows][nsplit] fp32
+ *   out: [rows][head_dim] fp32 or bf16; lse_out: [rows] or NULL.
+ */
+wmtp_status wmtp_splitkv_combine(int32_t rows, int32_t head_dim, int32_t nsplit,
+                                 const float* part_o, const float* part_lse, void* out,
+                                 int32_t out_fp32, float* lse_out, void* stream);
+
+/*
+ * wmtp_paged_write -- write new tokens' K/V into a paged cache.
+ * Support call (the append half of a decode step: the draft writes one token
+ * per draft forward, a verify layer writes its gamma+1 tokens).  For each
+ * sequence b and j < n_new: position pos0[b]+j goes to page
+ * page_table[b][(pos0[b]+j)/P], row (pos0[b]+j)%P.  kv->kv_len is not read or
+ * changed.
+ *   pos0: [batch] int32; k_new, v_new: [batch][n_new][Hkv][D] bf16.
+ */
+wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmtp_paged_kv* kv,
+                             const int32_t* pos0, int32_t n_new, const void* k_new,
+                             const void* v_new, int32_t* status_word, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WMTP_H_ */
