@@ -151,7 +151,7 @@ def workspace_bytes(kind: str, p: L.Params, batch: int, num_q: int = 1, max_page
     lib = L.load()
     size = c_size_t(0)
     if kind == "windowed":
-        desc = L.RingDesc(1, 1, 1, 1, 1, 1, 1, 1, batch)
+        desc = L.RingDesc(256, 256, 256, 256, 256, 256, 256, 256, batch)  # sizes only: never dereferenced
         L.check(kind, lib.wmtp_draft_attn_windowed(byref(p), None, byref(desc), None, 1, None, None,
                                                    byref(size), None, None))
     else:

@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  // let the dependent combine kernel get scheduled while this grid runs; it
+  // waits in-kernel until this grid has finished and its writes are visible
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // =================================================================== producer
   if (warp == kProducerWarp) {

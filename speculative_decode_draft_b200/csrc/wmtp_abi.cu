@@ -179,14 +179,26 @@ wmtp_status launch_decode(int D, int NT, const CUtensorMap& tk, const CUtensorMa
   return WMTP_ERR_UNSUPPORTED;
 }
 
+// `after_decode`: launched right behind a decode kernel on the same stream, as
+// its programmatic dependent (the combine waits in-kernel for the partials).
 wmtp_status launch_combine(int rows, int D, int nsplit, const float* po, const float* pl, void* out,
-                           int out_fp32, float* lse_out, cudaStream_t st) {
+                           int out_fp32, float* lse_out, cudaStream_t st, bool after_decode) {
   if (rows <= 0) return WMTP_OK;
-  if (out_fp32)
-    splitkv_combine_kernel<true><<<rows, kCombineThreads, 0, st>>>(po, pl, nsplit, D, out, lse_out);
-  else
-    splitkv_combine_kernel<false><<<rows, kCombineThreads, 0, st>>>(po, pl, nsplit, D, out, lse_out);
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(rows, (D + kCombineCols - 1) / kCombineCols, 1);
+  cfg.blockDim = dim3(kCombineThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_decode ? 1 : 0;
+  cudaError_t e = out_fp32 ? cudaLaunchKernelEx(&cfg, splitkv_combine_kernel<true>, po, pl, nsplit, D, out, lse_out)
+                           : cudaLaunchKernelEx(&cfg, splitkv_combine_kernel<false>, po, pl, nsplit, D, out,
+                                                lse_out);
+  return e == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
 }
 
 // Shared tail of the three attention entry points.
@@ -225,7 +237,7 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
   s = launch_decode<RING>(D, NT, *tk, *tv, a, B, st);
   if (s != WMTP_OK) return s;
   return launch_combine(static_cast<int>(rows_total), D, pl.nsplit, a.part_o, a.part_lse, out, out_fp32,
-                        lse_out, st);
+                        lse_out, st, true);
 }
 
 wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, const void* q,
@@ -410,11 +422,11 @@ wmtp_status wmtp_splitkv_combine(int32_t rows, int32_t head_dim, int32_t nsplit,
                                  const float* part_lse, void* out, int32_t out_fp32, float* lse_out,
                                  void* stream) {
   if (rows < 0 || nsplit <= 0) return WMTP_ERR_INVALID_ARG;
-  if (head_dim <= 0 || head_dim % 4 != 0 || head_dim > 4 * kCombineThreads) return WMTP_ERR_UNSUPPORTED;
+  if (head_dim <= 0 || head_dim % 4 != 0 || head_dim > 4096) return WMTP_ERR_UNSUPPORTED;
   if (rows > 0 && (part_o == nullptr || part_lse == nullptr || out == nullptr)) return WMTP_ERR_INVALID_ARG;
   if (!aligned(part_o, 16) || !aligned(out, 16)) return WMTP_ERR_INVALID_ARG;
   return launch_combine(rows, head_dim, nsplit, part_o, part_lse, out, out_fp32, lse_out,
-                        static_cast<cudaStream_t>(stream));
+                        static_cast<cudaStream_t>(stream), false);
 }
 
 wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmtp_paged_kv* kv,

@@ -112,7 +112,8 @@ def test_ring_calls_reject_bad_params(lib):
 
 def test_combine_and_paged_write_reject_bad_args(lib):
     assert lib.wmtp_splitkv_combine(4, 256, 0, None, None, None, 1, None, None) == L.WMTP_ERR_INVALID_ARG
-    assert lib.wmtp_splitkv_combine(4, 1024, 2, None, None, None, 1, None, None) == L.WMTP_ERR_UNSUPPORTED
+    assert lib.wmtp_splitkv_combine(4, 6, 2, None, None, None, 1, None, None) == L.WMTP_ERR_UNSUPPORTED
+    assert lib.wmtp_splitkv_combine(4, 8192, 2, None, None, None, 1, None, None) == L.WMTP_ERR_UNSUPPORTED
     assert lib.wmtp_splitkv_combine(4, 256, 2, None, None, None, 1, None, None) == L.WMTP_ERR_INVALID_ARG
     assert lib.wmtp_splitkv_combine(0, 256, 2, None, None, None, 1, None, None) == 0
     desc = L.PagedKVDesc(None, None, 8, None, 8, None)

@@ -89,7 +89,13 @@ def test_draft_full_bf16_output_within_one_ulp():
     assert out.dtype == torch.bfloat16
     kp, vp, pt, ln = _oracle_pools(kv)
     ref, _ = oracle.draft_attn_full(f64(q), kp, vp, pt, ln, 64, 1 / 16)
-    assert bf16_ulp_diff(out, ref) <= 1
+    # bf16 output = RNE(fp32 result): |out - ref| <= 2^-8 |ref| + the fp32
+    # error.  Near zero (cancellation) that fp32 error spans many bf16 ulps,
+    # so the one-ulp check applies only where |ref| >= 1e-2.
+    o = f64(out)
+    assert np.all(np.abs(o - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+    big = np.abs(ref) >= 1e-2
+    assert bf16_ulp_diff(out[torch.from_numpy(big).to(out.device)], ref[big]) <= 1
 
 
 def test_custom_softmax_scale():
