@@ -238,6 +238,34 @@ wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmt
                              const int32_t* pos0, int32_t n_new, const void* k_new,
                              const void* v_new, int32_t* status_word, void* stream);
 
+/*
+ * wmtp_draft_attn_full_noalloc -- wmtp_draft_attn_full without a workspace.
+ * The paper has no counterpart to this call; it exists for callers that
+ * cannot allocate device memory for the split-KV scratch: runtimes that plan
+ * all device memory before serving starts and forbid later allocations, and
+ * plugin hosts whose kernel interface passes only inputs and outputs.
+ *
+ * Same arguments, semantics and results as wmtp_draft_attn_full, minus the
+ * workspace pair.  The partial results go to one fixed device array of
+ * WMTP_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads the
+ * library holds that array until the process exits.  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current).  Make that first call before any
+ *     stream capture.
+ *   - A call whose scratch would exceed WMTP_NOALLOC_SCRATCH_BYTES returns
+ *     WMTP_ERR_WORKSPACE and launches nothing (the size is the one that
+ *     wmtp_draft_attn_full reports in *workspace_bytes).
+ *   - All calls share the array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero: every call overwrites each
+ *     partial it reads.  Calls that overlap on the GPU (different streams,
+ *     no ordering between them) race on the array and give wrong results.
+ */
+#define WMTP_NOALLOC_SCRATCH_BYTES (4u << 20)
+wmtp_status wmtp_draft_attn_full_noalloc(const wmtp_params* params, int32_t batch, const void* q,
+                                         const wmtp_paged_kv* kv, void* out, int32_t out_fp32,
+                                         float* lse_out, int32_t* status_word, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,11 @@ EXPORTS = (
     "wmtp_verify_attn",
     "wmtp_splitkv_combine",
     "wmtp_paged_write",
+    "wmtp_draft_attn_full_noalloc",
 )
+
+# Size of the fixed scratch array behind wmtp_draft_attn_full_noalloc.
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class Params(ctypes.Structure):
@@ -126,6 +130,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.wmtp_paged_write.restype = c_int32
     lib.wmtp_paged_write.argtypes = [PP, c_int32, PK, c_void_p, c_int32, c_void_p, c_void_p, i32p,
                                      c_void_p]
+    lib.wmtp_draft_attn_full_noalloc.restype = c_int32
+    lib.wmtp_draft_attn_full_noalloc.argtypes = [PP, c_int32, c_void_p, PK, c_void_p, c_int32, c_void_p,
+                                                 i32p, c_void_p]
     if path is None:
         _lib = lib
     return lib

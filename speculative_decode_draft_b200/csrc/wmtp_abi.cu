@@ -450,3 +450,50 @@ wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmt
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of wmtp_draft_attn_full.
+//
+// Some callers cannot hand this library a workspace: runtimes that plan every
+// device allocation up front and forbid new ones once serving starts, and
+// plugin hosts whose kernel interface passes only inputs and outputs.  For
+// them the split-KV partials live in the fixed array below instead of a
+// caller-provided buffer.  Every GPU that loads this library holds the array
+// until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t wmtp_noalloc_scratch[WMTP_NOALLOC_SCRATCH_BYTES];
+
+namespace wmtp {
+namespace {
+
+// Device address of the array on each device.  In host code the array's name
+// is only a host-side stand-in, so the real address is fetched once per
+// device, with that device current, and passed to the kernels.
+void* g_noalloc_ptr[kMaxDevices] = {};
+cudaError_t g_noalloc_err[kMaxDevices] = {};
+std::once_flag g_noalloc_once[kMaxDevices];
+
+}  // namespace
+}  // namespace wmtp
+
+extern "C" wmtp_status wmtp_draft_attn_full_noalloc(const wmtp_params* params, int32_t batch, const void* q,
+                                                    const wmtp_paged_kv* kv, void* out, int32_t out_fp32,
+                                                    float* lse_out, int32_t* status_word, void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
+  std::call_once(g_noalloc_once[dev], [dev]() {
+    void* ptr = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, wmtp_noalloc_scratch);
+    g_noalloc_ptr[dev] = ptr;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return WMTP_ERR_CUDA;
+  size_t need = 0;
+  wmtp_status s = paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, nullptr, &need,
+                                  status_word, stream);
+  if (s != WMTP_OK) return s;
+  if (need > static_cast<size_t>(WMTP_NOALLOC_SCRATCH_BYTES)) return WMTP_ERR_WORKSPACE;
+  if (batch == 0) return WMTP_OK;
+  size_t have = WMTP_NOALLOC_SCRATCH_BYTES;
+  return paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, g_noalloc_ptr[dev], &have,
+                         status_word, stream);
+}
