@@ -1,0 +1,445 @@
+// Verify attention on the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+//
+// The target verifies gamma+1 draft tokens with causal attention over its
+// full paged KV ("Windowed-MTP ..." arxivlens view, Abstract: verification
+// stays full-context).  All rows = (gamma+1) x G query heads of one KV head
+// share each K/V byte; with G = 8 that is 16..64 rows against every token.
+//
+// Per CTA = (split, KV head, sequence), head_dim 256, 64-token tiles, with
+// the rows as the MMA M dimension (padded to 128) and everything but K and V
+// kept in tensor memory (512 columns x 128 lanes):
+//   columns   0..127  Q            bf16 pairs, the A operand of S = Q K^T
+//   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax the
+//                                  same columns hold P as bf16 hi (0..31) and
+//                                  lo (32..63) pairs, the A operand of P V
+//   columns 256..511  O            fp32 output accumulator, 256 head dims
+// Row r of the block sits in TMEM lane 32 (r % 4) + r / 4, so the rows spread
+// over the four lane quadrants and each softmax warp owns a quarter of them.
+//
+// Roles: warp 0 streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
+// into a STAGES-deep shared-memory ring with TMA; warp 1 allocates the tensor
+// memory and one lane issues every MMA (S = Q K^T as M=128, N=64 with K from
+// shared memory, K-major; O += P V as M=128, N=256 with V read MN-major
+// straight from the TMA tile); warps 2..5 run the softmax, one thread per
+// row: the row's scores come out of TMEM, the maximum and sum are taken
+// inside the thread, and P goes back into TMEM as bf16 hi + lo
+// (|p - hi - lo| <= 2^-16 p, so the PV product keeps about fp32 weight
+// precision).  The reference maximum of a row is raised only when the tile
+// maximum exceeds it by more than 2^8 (weights then stay below 256), and only
+// then is that row of O rescaled in TMEM, after the previous PV completed.
+//
+// Every mbarrier wait is bounded; a wait that gives up raises
+// WMTP_DEV_TIMEOUT, stops the pipeline, waits (bounded) for the MMAs already
+// issued and frees the tensor memory before the CTA exits.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "decode_attn.cuh"
+#include "ptx.cuh"
+
+namespace wmtp {
+
+constexpr int kTcThreads = 192;       // producer, MMA, 4 softmax warps
+constexpr int kBarTmem = 3;           // named barrier: MMA + softmax warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColQ = 0;
+constexpr uint32_t kColS = 128;
+constexpr uint32_t kColO = 256;
+constexpr float kRescaleLog2 = 8.f;   // lazy rescale threshold (log2 units)
+
+template <int STAGES>
+struct TcPlan {
+  static constexpr int kChunkBytes = 64 * 128;           // 64 tokens x 128 B
+  static constexpr int kTileBytes = 4 * kChunkBytes;      // one K or V tile, D = 256
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffBar = STAGES * kStageBytes;
+  // kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, mma_final
+  static constexpr int kNumBars = 2 * STAGES + 6;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, stage flags
+  static constexpr int kBytes = kOffMisc + 8 + 4 * STAGES;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+constexpr int kTcStages = 3;
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag != 0) return false;
+    if (clock64() - t0 > ptx::kWaitLimitCycles) return false;
+  }
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                     const DecodeArgs a) {
+  using Plan = TcPlan<STAGES>;
+  constexpr int D = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t bar0 = sbase + Plan::kOffBar;
+  const uint32_t bar_kv_full = bar0;
+  const uint32_t bar_kv_empty = bar0 + 8 * STAGES;
+  const uint32_t bar_s_full = bar0 + 16 * STAGES;
+  const uint32_t bar_p_full = bar_s_full + 16;
+  const uint32_t bar_o_done = bar_p_full + 16;
+  const uint32_t bar_final = bar_o_done + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
+  volatile int* stage_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 8);
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- token range of this split
+  int n_tok = a.kv_len[b];
+  if (n_tok != 0 && (n_tok < a.num_q || n_tok > a.max_pages * a.page_size)) {
+    if (threadIdx.x == 0 && split == 0 && kvh == 0) set_status(a.status, kDevLenOob);
+    n_tok = 0;
+  }
+  const int ntiles = (n_tok + kTileTokens - 1) / kTileTokens;
+  const int tps = (ntiles + a.nsplit - 1) / a.nsplit;
+  const int t_begin = min(split * tps, ntiles);
+  const int t_end = min(t_begin + tps, ntiles);
+  const int my_tiles = t_end - t_begin;
+
+  // ---- set-up: barriers and tensor memory
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(bar_kv_full + 8 * s, 1);
+      ptx::mbar_init(bar_kv_empty + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar_s_full + 8 * i, 1);
+      ptx::mbar_init(bar_p_full + 8 * i, 4);
+    }
+    ptx::mbar_init(bar_o_done, 1);
+    ptx::mbar_init(bar_final, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // softmax-thread identity: TMEM lane m = 32 q + lane holds row 4 lane + q
+  const int q = warp & 3;
+  const int row = 4 * lane + q;
+  const bool row_active = warp >= 2 && lane < 16 && row < a.rows;
+  const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+
+  if (warp >= 2) {
+    // Q row into TMEM columns 0..127 (bf16 pairs), zeros for padding rows
+    const __nv_bfloat16* src =
+        row_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
+                   : nullptr;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row_active) v = *reinterpret_cast<const uint4*>(src + 64 * c + 8 * j);
+        w[4 * j] = v.x;
+        w[4 * j + 1] = v.y;
+        w[4 * j + 2] = v.z;
+        w[4 * j + 3] = v.w;
+      }
+      tc::tmem_st32(tmem_base + lane_addr + kColQ + 32 * c, w);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // =================================================================== producer
+  if (warp == 0) {
+    if (lane == 0 && my_tiles > 0) {
+      ptx::prefetch_tmap(&tmap_k);
+      ptx::prefetch_tmap(&tmap_v);
+      const uint64_t pol = ptx::policy_evict_first();
+      const int box_rows = min(a.page_size, kTileTokens);
+      const int boxes = kTileTokens / box_rows;
+      const int oob_z = a.num_pages * a.Hkv;  // past the tensor: zero fill
+      for (int k = 0; k < my_tiles; ++k) {
+        const int stage = k % STAGES;
+        if (!tc_wait(bar_kv_empty + 8 * stage, ((k / STAGES) & 1) ^ 1, abort_flag)) {
+          if (*abort_flag == 0) set_status(a.status, kDevTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        const int tok0 = (t_begin + k) * kTileTokens;
+        const uint32_t kdst = sbase + Plan::kOffK + stage * Plan::kStageBytes;
+        const uint32_t vdst = kdst + Plan::kTileBytes;
+        const uint32_t fb = bar_kv_full + 8 * stage;
+        int zs[4], ys[4];
+        int valid = 1;
+        for (int j = 0; j < boxes; ++j) {
+          const int tok = tok0 + j * box_rows;
+          zs[j] = oob_z;
+          ys[j] = 0;
+          if (tok >= n_tok) continue;
+          const int lp = tok / a.page_size;
+          const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + lp];
+          if (pg < 0 || pg >= a.num_pages) {
+            valid = 0;
+          } else {
+            zs[j] = pg * a.Hkv + kvh;
+            ys[j] = tok - lp * a.page_size;
+          }
+        }
+        if (!valid) set_status(a.status, kDevPageOob);
+        stage_flag[stage] = valid;
+        ptx::mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+        for (int j = 0; j < boxes; ++j) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t off = c * Plan::kChunkBytes + j * box_rows * 128;
+            ptx::tma_load_3d(kdst + off, &tmap_k, fb, c * 64, ys[j], zs[j], pol);
+            ptx::tma_load_3d(vdst + off, &tmap_v, fb, c * 64, ys[j], zs[j], pol);
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // =================================================================== MMA issuer
+  if (warp == 1) {
+    if (lane == 0 && my_tiles > 0) {
+      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(128, 64, 0, 0);   // A (Q, TMEM), B (K) K-major
+      constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(128, 256, 0, 1);  // A (P, TMEM), B (V) MN-major
+      // descriptor start addresses are in 16-byte units in the low bits, so
+      // moving an operand by n bytes adds n >> 4 to the descriptor
+      const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
+      const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK + Plan::kTileBytes, Plan::kChunkBytes, 1024);
+      auto issue_qk = [&](int k) {
+        const uint64_t kd = k_desc0 + (static_cast<uint64_t>((k % STAGES) * Plan::kStageBytes) >> 4);
+        const uint32_t d_tmem = tmem_base + kColS + (k & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
+          tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(bar_s_full + 8 * (k & 1));
+      };
+      bool ok = tc_wait(bar_kv_full, 0, abort_flag);
+      if (ok) {
+        tc::fence_after_sync();
+        issue_qk(0);
+      }
+      for (int k = 0; ok && k < my_tiles; ++k) {
+        if (k + 1 < my_tiles) {
+          // the S/P buffer of tile k+1 last held P(k-1), read by PV(k-1),
+          // which was issued earlier and runs first
+          ok = tc_wait(bar_kv_full + 8 * ((k + 1) % STAGES), ((k + 1) / STAGES) & 1, abort_flag);
+          if (!ok) break;
+          tc::fence_after_sync();
+          issue_qk(k + 1);
+        }
+        ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint64_t vd = v_desc0 + (static_cast<uint64_t>((k % STAGES) * Plan::kStageBytes) >> 4);
+        const uint32_t p_tmem = tmem_base + kColS + (k & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+          const uint64_t bd = vd + (static_cast<uint32_t>(kk * 2048) >> 4);
+          tc::mma_ts(tmem_base + kColO, p_tmem + 8 * kk, bd, kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(tmem_base + kColO, p_tmem + 32 + 8 * kk, bd, kIdescPV, 1u);
+        }
+        tc::commit(bar_kv_empty + 8 * (k % STAGES));
+        tc::commit(bar_o_done);
+      }
+      if (!ok) {
+        if (*abort_flag == 0) set_status(a.status, kDevTimeout);
+        *abort_flag = 1;
+      }
+      // wait (bounded) until every MMA issued here has completed, so the
+      // tensor memory is never freed under a running MMA
+      tc::commit(bar_final);
+      if (!ptx::mbar_wait(bar_final, 0)) set_status(a.status, kDevTimeout);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================= softmax
+    const int lim = row_active ? n_tok - a.num_q + row / a.G + 1 : n_tok;  // causal limit of this row
+    const int first_masked_tok = n_tok - a.num_q + 1;
+    float m_ref = -INFINITY;  // reference maximum (log2 units)
+    float l_run = 0.f;
+    bool failed = false;
+
+    for (int k = 0; k < my_tiles; ++k) {
+      const int stage = k % STAGES;
+      const int sb = k & 1;
+      const bool ok = __all_sync(0xffffffffu, tc_wait(bar_kv_full + 8 * stage, (k / STAGES) & 1, abort_flag) &&
+                                                  tc_wait(bar_s_full + 8 * sb, (k >> 1) & 1, abort_flag));
+      if (!ok) {
+        failed = true;
+        break;  // this warp stops; the MMA warp times out or sees the abort
+      }
+      tc::fence_after_sync();
+      const int tok0 = (t_begin + k) * kTileTokens;
+      const bool tile_ok = stage_flag[stage] != 0;
+      const uint32_t s_addr = tmem_base + lane_addr + kColS + sb * 64;
+
+      uint32_t sraw[64];
+      tc::tmem_ld32(s_addr, sraw);
+      tc::tmem_ld32(s_addr + 32, sraw + 32);
+      float x[64];
+      float mx = -INFINITY;
+      if (tok0 + kTileTokens <= first_masked_tok) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          x[j] = tile_ok ? __uint_as_float(sraw[j]) * a.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[j]);
+        }
+      } else {  // tile holding the causal tail and/or the end of the sequence
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const int t = tok0 + j;
+          x[j] = (tile_ok && t < lim && t < n_tok) ? __uint_as_float(sraw[j]) * a.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[j]);
+        }
+      }
+      // raise the reference maximum only when the tile exceeds it by more
+      // than 2^8; rows whose reference moved rescale their O row and sum
+      float alpha = 1.f;
+      bool moved = false;
+      if (mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx != -INFINITY)) {
+        alpha = (m_ref == -INFINITY) ? 0.f : ptx::ex2(m_ref - mx);
+        moved = m_ref != -INFINITY;
+        m_ref = mx;
+      }
+      const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
+      if (__any_sync(0xffffffffu, moved)) {
+        // PV(k-1) must have finished before O is rewritten.  S(k) arriving
+        // implies PV(k-2) completed (issued before QK(k)), so the pending
+        // o_done phase is PV(k-1)'s and a parity wait is unambiguous.
+        if (!__all_sync(0xffffffffu, tc_wait(bar_o_done, (k - 1) & 1, abort_flag))) {
+          failed = true;
+          break;
+        }
+        tc::fence_after_sync();
+        const float f = moved ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(tmem_base + lane_addr + kColO + 32 * c, o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+          tc::tmem_st32(tmem_base + lane_addr + kColO + 32 * c, o);
+        }
+      }
+      // P = 2^(x - base) as bf16 hi + lo pairs, back into the S columns
+      float sum = 0.f;
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float p0 = ptx::ex2(x[2 * j] - base);  // 2^-inf = 0 for masked entries
+        const float p1 = ptx::ex2(x[2 * j + 1] - base);
+        sum += p0 + p1;
+        hi[j] = ptx::pack_bf16x2(p0, p1);
+        lo[j] = ptx::pack_bf16x2(p0 - ptx::bf16lo_to_f32(hi[j]), p1 - ptx::bf16hi_to_f32(hi[j]));
+      }
+      l_run = l_run * alpha + sum;
+      tc::tmem_st32(s_addr, hi);
+      tc::tmem_st32(s_addr + 32, lo);
+
+      // zero V rows past the valid length (tail tile only; rows r with
+      // r % 4 == q by this warp)
+      if (tok0 + kTileTokens > n_tok) {
+        const uint32_t vst = sbase + Plan::kOffK + stage * Plan::kStageBytes + Plan::kTileBytes;
+        const int r0 = max(n_tok - tok0, 0);
+        for (int u = lane; u < (kTileTokens - r0) * (D / 8); u += 32) {
+          const int r = r0 + u / (D / 8);
+          const int j = u % (D / 8);
+          if ((r & 3) != q) continue;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
+                           vst + (j >> 3) * Plan::kChunkBytes + r * 128 + ((j & 7) << 4)),
+                       "r"(0)
+                       : "memory");
+        }
+        ptx::fence_proxy_async_smem();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_p_full + 8 * sb);
+    }
+
+    // ---- finish: normalised partial output and log-sum-exp of this row
+    if (!failed && my_tiles > 0) {
+      // o_done completes once per PV.  When the last S arrived, PV(n-3) had
+      // completed (it was issued before that QK) but PV(n-2) may not have, so
+      // wait for the phases of PV(n-2) and PV(n-1) in turn: a parity wait
+      // only tells the pending phase from the one just before it.
+      bool done = true;
+      if (my_tiles >= 2) done = tc_wait(bar_o_done, (my_tiles - 2) & 1, abort_flag);
+      done = done && tc_wait(bar_o_done, (my_tiles - 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, done)) failed = true;
+      tc::fence_after_sync();
+    }
+    failed = __any_sync(0xffffffffu, failed);
+    if (failed) {
+      if (lane == 0) set_status(a.status, kDevTimeout);
+      *abort_flag = 1;
+    }
+    const float inv = (l_run > 0.f && !failed) ? 1.f / l_run : 0.f;
+    const size_t grow =
+        row_active ? (static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G : 0;
+    float* dst = a.part_o + (grow * a.nsplit + split) * D;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      uint32_t o[32];
+      if (my_tiles > 0 && !failed) {
+        tc::tmem_ld32(tmem_base + lane_addr + kColO + 32 * c, o);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = 0u;
+      }
+      if (row_active) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + 32 * c + j) =
+              make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
+                          __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+      }
+    }
+    if (row_active) {
+      // m_ref is in log2 units of the scaled score
+      a.part_lse[grow * a.nsplit + split] =
+          (l_run > 0.f && !failed) ? m_ref * 0.69314718055994531f + logf(l_run) : -INFINITY;
+    }
+    tc::fence_before_sync();
+  }
+
+  // ---- every MMA has completed (the MMA lane waited for its final commit);
+  // free the tensor memory
+  ptx::named_bar_sync(kBarTmem, 160);
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace wmtp

@@ -14,6 +14,7 @@
 #include "combine.cuh"
 #include "decode_attn.cuh"
 #include "ring.cuh"
+#include "verify_tc.cuh"
 #include "wmtp.h"
 
 namespace wmtp {
@@ -179,6 +180,27 @@ wmtp_status launch_decode(int D, int NT, const CUtensorMap& tk, const CUtensorMa
   return WMTP_ERR_UNSUPPORTED;
 }
 
+wmtp_status launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
+                             cudaStream_t st) {
+  constexpr int alloc = TcPlan<kTcStages>::kAlloc;
+  static_assert(alloc <= kSmemLimit, "shared-memory plan exceeds the sm_100 per-block limit");
+  auto kern = verify_tc_kernel<kTcStages>;
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc) != cudaSuccess)
+      return WMTP_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  dim3 grid(a.nsplit, a.Hkv, B);
+  kern<<<grid, kTcThreads, alloc, st>>>(tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+}
+
+// Verify blocks of head_dim 256 with 9..64 query rows run on tcgen05.
+bool use_verify_tc(int D, int num_q, int rows) { return D == 256 && num_q >= 2 && rows >= 9 && rows <= 64; }
+
 // `after_decode`: launched right behind a decode kernel on the same stream, as
 // its programmatic dependent (the combine waits in-kernel for the partials).
 wmtp_status launch_combine(int rows, int D, int nsplit, const float* po, const float* pl, void* out,
@@ -234,7 +256,10 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
   a.scale_log2 = scale_log2(p);
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_lse);
-  s = launch_decode<RING>(D, NT, *tk, *tv, a, B, st);
+  if (!RING && use_verify_tc(D, num_q, rows))
+    s = launch_verify_tc(*tk, *tv, a, B, st);
+  else
+    s = launch_decode<RING>(D, NT, *tk, *tv, a, B, st);
   if (s != WMTP_OK) return s;
   return launch_combine(static_cast<int>(rows_total), D, pl.nsplit, a.part_o, a.part_lse, out, out_fp32,
                         lse_out, st, true);
