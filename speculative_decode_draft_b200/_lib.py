@@ -25,6 +25,7 @@ DEV_LEN_OOB = 0x2
 DEV_RING_STATE = 0x4
 DEV_UNDO_FULL = 0x8
 DEV_TIMEOUT = 0x10
+DEV_V_RANGE = 0x20
 
 EXPORTS = (
     "wmtp_status_string",

@@ -59,6 +59,7 @@ constexpr int kDevLenOob = 0x2;
 constexpr int kDevRingState = 0x4;
 constexpr int kDevUndoFull = 0x8;
 constexpr int kDevTimeout = 0x10;
+constexpr int kDevVRange = 0x20;
 
 struct DecodeArgs {
   const __nv_bfloat16* q;  // [B][num_q][Hq][D]

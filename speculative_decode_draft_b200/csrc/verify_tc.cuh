@@ -9,24 +9,35 @@
 // the rows as the MMA M dimension (padded to 128) and everything but K and V
 // kept in tensor memory (512 columns x 128 lanes):
 //   columns   0..127  Q            bf16 pairs, the A operand of S = Q K^T
-//   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax the
-//                                  same columns hold P as bf16 hi (0..31) and
-//                                  lo (32..63) pairs, the A operand of P V
+//   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax
+//                                  columns 0..31 of the buffer hold P as fp16
+//                                  pairs, the A operand of P V
 //   columns 256..511  O            fp32 output accumulator, 256 head dims
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4, so the rows spread
 // over the four lane quadrants and each softmax warp owns a quarter of them.
 //
 // Roles: warp 0 streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
-// into a STAGES-deep shared-memory ring with TMA; warp 1 allocates the tensor
+// into two STAGES-deep shared-memory rings with TMA, one lane per ring: a K
+// tile is released as soon as its S = Q K^T has completed, a V tile only
+// after its O += P V, so K loads run ahead of the softmax instead of waiting
+// for the slower PV of the same tile; warp 1 allocates the tensor
 // memory and one lane issues every MMA (S = Q K^T as M=128, N=64 with K from
 // shared memory, K-major; O += P V as M=128, N=256 with V read MN-major
 // straight from the TMA tile); warps 2..5 run the softmax, one thread per
 // row: the row's scores come out of TMEM, the maximum and sum are taken
-// inside the thread, and P goes back into TMEM as bf16 hi + lo
-// (|p - hi - lo| <= 2^-16 p, so the PV product keeps about fp32 weight
-// precision).  The reference maximum of a row is raised only when the tile
-// maximum exceeds it by more than 2^8 (weights then stay below 256), and only
-// then is that row of O rescaled in TMEM, after the previous PV completed.
+// inside the thread, and P goes back into TMEM in fp16; warps 6..9 convert
+// each landed V tile in place from bf16 to fp16 (and zero its rows past the
+// sequence end).  The value product is therefore fp16 x fp16 -> fp32: P
+// carries a relative rounding of at most 2^-11 (bf16 would give 2^-8 and miss
+// a 1e-3 relative-L2 bound), and V is exact for every |v| < 2^16 (below 2^-17
+// the absolute error stays under 2^-25); a larger |v| saturates and raises
+// WMTP_DEV_V_RANGE.  On sm_100 a tcgen05.mma of these shapes costs a fixed
+// ~100 cycles, so one fp16 MMA per 16 tokens instead of a bf16 hi + lo pair
+// is what keeps the block under the HBM time of a tile.
+// The reference maximum of a row is raised only when the tile maximum
+// exceeds it by more than 2^8 (weights then stay below 256, well inside
+// fp16), and only then is that row of O rescaled in TMEM, after the previous
+// PV completed.
 //
 // Every mbarrier wait is bounded; a wait that gives up raises
 // WMTP_DEV_TIMEOUT, stops the pipeline, waits (bounded) for the MMAs already
@@ -42,7 +53,7 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 192;       // producer, MMA, 4 softmax warps
+constexpr int kTcThreads = 320;       // producers, MMA, 4 softmax warps, 4 V converter warps
 constexpr int kBarTmem = 3;           // named barrier: MMA + softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;
@@ -57,10 +68,11 @@ struct TcPlan {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kOffK = 0;
   static constexpr int kOffBar = STAGES * kStageBytes;
-  // kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, mma_final
-  static constexpr int kNumBars = 2 * STAGES + 6;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, stage flags
-  static constexpr int kBytes = kOffMisc + 8 + 4 * STAGES;
+  // k_full[S], k_empty[S], v_full[S], v_empty[S], v_ready[S], s_full[2],
+  // p_full[2], o_done, mma_final
+  static constexpr int kNumBars = 5 * STAGES + 6;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort
+  static constexpr int kBytes = kOffMisc + 8;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -89,15 +101,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = ptx::smem_addr(smem);
   const uint32_t bar0 = sbase + Plan::kOffBar;
-  const uint32_t bar_kv_full = bar0;
-  const uint32_t bar_kv_empty = bar0 + 8 * STAGES;
-  const uint32_t bar_s_full = bar0 + 16 * STAGES;
+  const uint32_t bar_k_full = bar0;
+  const uint32_t bar_k_empty = bar0 + 8 * STAGES;
+  const uint32_t bar_v_full = bar0 + 16 * STAGES;
+  const uint32_t bar_v_empty = bar0 + 24 * STAGES;
+  const uint32_t bar_v_ready = bar0 + 32 * STAGES;
+  const uint32_t bar_s_full = bar0 + 40 * STAGES;
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_o_done = bar_p_full + 16;
   const uint32_t bar_final = bar_o_done + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
-  volatile int* stage_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 8);
 
   const int split = blockIdx.x;
   const int kvh = blockIdx.y;
@@ -120,8 +134,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // ---- set-up: barriers and tensor memory
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(bar_kv_full + 8 * s, 1);
-      ptx::mbar_init(bar_kv_empty + 8 * s, 1);
+      ptx::mbar_init(bar_k_full + 8 * s, 1);
+      ptx::mbar_init(bar_k_empty + 8 * s, 1);
+      ptx::mbar_init(bar_v_full + 8 * s, 1);
+      ptx::mbar_init(bar_v_empty + 8 * s, 1);
+      ptx::mbar_init(bar_v_ready + 8 * s, 4);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar_s_full + 8 * i, 1);
@@ -144,10 +161,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // softmax-thread identity: TMEM lane m = 32 q + lane holds row 4 lane + q
   const int q = warp & 3;
   const int row = 4 * lane + q;
-  const bool row_active = warp >= 2 && lane < 16 && row < a.rows;
+  const bool row_active = warp >= 2 && warp < 6 && lane < 16 && row < a.rows;
   const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
 
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     // Q row into TMEM columns 0..127 (bf16 pairs), zeros for padding rows
     const __nv_bfloat16* src =
         row_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
@@ -172,26 +189,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::fence_after_sync();
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // =================================================================== producer
+  // =================================================================== producers
+  // lane 0 loads K tiles, lane 1 loads V tiles; each has its own ring
   if (warp == 0) {
-    if (lane == 0 && my_tiles > 0) {
-      ptx::prefetch_tmap(&tmap_k);
-      ptx::prefetch_tmap(&tmap_v);
+    if (lane < 2 && my_tiles > 0) {
+      const bool is_k = lane == 0;
+      const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+      ptx::prefetch_tmap(tmap);
       const uint64_t pol = ptx::policy_evict_first();
       const int box_rows = min(a.page_size, kTileTokens);
       const int boxes = kTileTokens / box_rows;
       const int oob_z = a.num_pages * a.Hkv;  // past the tensor: zero fill
+      const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
+      const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
+      const uint32_t ring = sbase + Plan::kOffK + (is_k ? 0 : Plan::kTileBytes);
       for (int k = 0; k < my_tiles; ++k) {
         const int stage = k % STAGES;
-        if (!tc_wait(bar_kv_empty + 8 * stage, ((k / STAGES) & 1) ^ 1, abort_flag)) {
+        if (!tc_wait(bar_empty + 8 * stage, ((k / STAGES) & 1) ^ 1, abort_flag)) {
           if (*abort_flag == 0) set_status(a.status, kDevTimeout);
           *abort_flag = 1;
           break;
         }
         const int tok0 = (t_begin + k) * kTileTokens;
-        const uint32_t kdst = sbase + Plan::kOffK + stage * Plan::kStageBytes;
-        const uint32_t vdst = kdst + Plan::kTileBytes;
-        const uint32_t fb = bar_kv_full + 8 * stage;
+        const uint32_t dst = ring + stage * Plan::kStageBytes;
+        const uint32_t fb = bar_full + 8 * stage;
         int zs[4], ys[4];
         int valid = 1;
         for (int j = 0; j < boxes; ++j) {
@@ -208,19 +229,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ys[j] = tok - lp * a.page_size;
           }
         }
-        if (!valid) set_status(a.status, kDevPageOob);
-        stage_flag[stage] = valid;
-        ptx::mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+        if (is_k && !valid) set_status(a.status, kDevPageOob);
+        ptx::mbar_arrive_expect_tx(fb, Plan::kTileBytes);
         for (int j = 0; j < boxes; ++j) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t off = c * Plan::kChunkBytes + j * box_rows * 128;
-            ptx::tma_load_3d(kdst + off, &tmap_k, fb, c * 64, ys[j], zs[j], pol);
-            ptx::tma_load_3d(vdst + off, &tmap_v, fb, c * 64, ys[j], zs[j], pol);
-          }
+          for (int c = 0; c < 4; ++c)
+            ptx::tma_load_3d(dst + c * Plan::kChunkBytes + j * box_rows * 128, tmap, fb, c * 64, ys[j], zs[j], pol);
         }
       }
     }
+    return;
+  }
+
+  // =================================================================== V converters
+  if (warp >= 6) {
+    const int cw = warp - 6;  // one 8 KB column chunk (64 head dims) of the V tile per warp
+    uint32_t vexp = 0;        // per-half maximum of the bf16 exponent fields seen
+    for (int k = 0; k < my_tiles; ++k) {
+      const int stage = k % STAGES;
+      if (!__all_sync(0xffffffffu, tc_wait(bar_v_full + 8 * stage, (k / STAGES) & 1, abort_flag))) {
+        if (lane == 0) set_status(a.status, kDevTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      const int tok0 = (t_begin + k) * kTileTokens;
+      const int rows_valid = min(kTileTokens, n_tok - tok0);
+      const uint32_t chunk = sbase + Plan::kOffK + stage * Plan::kStageBytes + Plan::kTileBytes +
+                             cw * Plan::kChunkBytes;
+#pragma unroll 4
+      for (int u = lane; u < Plan::kChunkBytes / 16; u += 32) {
+        const uint32_t addr = chunk + 16 * u;
+        uint4 w;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                     : "r"(addr));
+        if (u / 8 < rows_valid) {  // 8 sixteen-byte units per 128-byte row
+          vexp = __vmaxu2(vexp, __vmaxu2(w.x & 0x7f807f80u, w.y & 0x7f807f80u));
+          vexp = __vmaxu2(vexp, __vmaxu2(w.z & 0x7f807f80u, w.w & 0x7f807f80u));
+          w.x = ptx::bf16x2_to_f16x2_sat(w.x);
+          w.y = ptx::bf16x2_to_f16x2_sat(w.y);
+          w.z = ptx::bf16x2_to_f16x2_sat(w.z);
+          w.w = ptx::bf16x2_to_f16x2_sat(w.w);
+        } else {  // past the end of the sequence: zero, so 0-weight rows add 0
+          w = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w.x), "r"(w.y), "r"(w.z),
+                     "r"(w.w)
+                     : "memory");
+      }
+      ptx::fence_proxy_async_smem();  // generic writes before the tensor core reads
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_v_ready + 8 * stage);
+    }
+    // a bf16 exponent field of 143 or more means |v| >= 2^16
+    if ((vexp & 0xffffu) >= (143u << 7) || (vexp >> 16) >= (143u << 7)) set_status(a.status, kDevVRange);
     return;
   }
 
@@ -228,7 +290,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 1) {
     if (lane == 0 && my_tiles > 0) {
       constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(128, 64, 0, 0);   // A (Q, TMEM), B (K) K-major
-      constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(128, 256, 0, 1);  // A (P, TMEM), B (V) MN-major
+      constexpr uint32_t kIdescPV = tc::idesc_f16_f32(128, 256, 0, 1);   // A (P, TMEM), B (V) MN-major, fp16
       // descriptor start addresses are in 16-byte units in the low bits, so
       // moving an operand by n bytes adds n >> 4 to the descriptor
       const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
@@ -242,8 +304,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
         }
         tc::commit(bar_s_full + 8 * (k & 1));
+        tc::commit(bar_k_empty + 8 * (k % STAGES));
       };
-      bool ok = tc_wait(bar_kv_full, 0, abort_flag);
+      bool ok = tc_wait(bar_k_full, 0, abort_flag);
       if (ok) {
         tc::fence_after_sync();
         issue_qk(0);
@@ -252,12 +315,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (k + 1 < my_tiles) {
           // the S/P buffer of tile k+1 last held P(k-1), read by PV(k-1),
           // which was issued earlier and runs first
-          ok = tc_wait(bar_kv_full + 8 * ((k + 1) % STAGES), ((k + 1) / STAGES) & 1, abort_flag);
+          ok = tc_wait(bar_k_full + 8 * ((k + 1) % STAGES), ((k + 1) / STAGES) & 1, abort_flag);
           if (!ok) break;
           tc::fence_after_sync();
           issue_qk(k + 1);
         }
-        ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag);
+        ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag) &&
+             tc_wait(bar_v_ready + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
         const uint64_t vd = v_desc0 + (static_cast<uint64_t>((k % STAGES) * Plan::kStageBytes) >> 4);
@@ -266,9 +330,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
           const uint64_t bd = vd + (static_cast<uint32_t>(kk * 2048) >> 4);
           tc::mma_ts(tmem_base + kColO, p_tmem + 8 * kk, bd, kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
-          tc::mma_ts(tmem_base + kColO, p_tmem + 32 + 8 * kk, bd, kIdescPV, 1u);
         }
-        tc::commit(bar_kv_empty + 8 * (k % STAGES));
+        tc::commit(bar_v_empty + 8 * (k % STAGES));
         tc::commit(bar_o_done);
       }
       if (!ok) {
@@ -292,15 +355,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int k = 0; k < my_tiles; ++k) {
       const int stage = k % STAGES;
       const int sb = k & 1;
-      const bool ok = __all_sync(0xffffffffu, tc_wait(bar_kv_full + 8 * stage, (k / STAGES) & 1, abort_flag) &&
-                                                  tc_wait(bar_s_full + 8 * sb, (k >> 1) & 1, abort_flag));
+      // S(k) complete implies K(k) landed.  (The K ring itself is not waited
+      // on here: its stage may already hold a later tile, so a parity wait on
+      // it would be ambiguous.)
+      const bool ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8 * sb, (k >> 1) & 1, abort_flag));
       if (!ok) {
         failed = true;
         break;  // this warp stops; the MMA warp times out or sees the abort
       }
       tc::fence_after_sync();
       const int tok0 = (t_begin + k) * kTileTokens;
-      const bool tile_ok = stage_flag[stage] != 0;
+      // a tile with a page outside the pool is skipped (the producers loaded
+      // zeros for it and raised WMTP_DEV_PAGE_OOB)
+      bool tile_ok = true;
+      for (int tok = tok0; tok < min(tok0 + kTileTokens, n_tok); tok += min(a.page_size, kTileTokens)) {
+        const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size];
+        tile_ok = tile_ok && pg >= 0 && pg < a.num_pages;
+      }
       const uint32_t s_addr = tmem_base + lane_addr + kColS + sb * 64;
 
       uint32_t sraw[64];
@@ -351,37 +422,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc::tmem_st32(tmem_base + lane_addr + kColO + 32 * c, o);
         }
       }
-      // P = 2^(x - base) as bf16 hi + lo pairs, back into the S columns
+      // P = 2^(x - base) as fp16 pairs, back into the S columns
       float sum = 0.f;
-      uint32_t hi[32], lo[32];
+      uint32_t ph[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float p0 = ptx::ex2(x[2 * j] - base);  // 2^-inf = 0 for masked entries
         const float p1 = ptx::ex2(x[2 * j + 1] - base);
         sum += p0 + p1;
-        hi[j] = ptx::pack_bf16x2(p0, p1);
-        lo[j] = ptx::pack_bf16x2(p0 - ptx::bf16lo_to_f32(hi[j]), p1 - ptx::bf16hi_to_f32(hi[j]));
+        ph[j] = ptx::pack_f16x2(p0, p1);
       }
       l_run = l_run * alpha + sum;
-      tc::tmem_st32(s_addr, hi);
-      tc::tmem_st32(s_addr + 32, lo);
+      tc::tmem_st32(s_addr, ph);
 
-      // zero V rows past the valid length (tail tile only; rows r with
-      // r % 4 == q by this warp)
-      if (tok0 + kTileTokens > n_tok) {
-        const uint32_t vst = sbase + Plan::kOffK + stage * Plan::kStageBytes + Plan::kTileBytes;
-        const int r0 = max(n_tok - tok0, 0);
-        for (int u = lane; u < (kTileTokens - r0) * (D / 8); u += 32) {
-          const int r = r0 + u / (D / 8);
-          const int j = u % (D / 8);
-          if ((r & 3) != q) continue;
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
-                           vst + (j >> 3) * Plan::kChunkBytes + r * 128 + ((j & 7) << 4)),
-                       "r"(0)
-                       : "memory");
-        }
-        ptx::fence_proxy_async_smem();
-      }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_p_full + 8 * sb);

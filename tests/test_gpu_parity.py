@@ -360,3 +360,16 @@ def test_workspace_query_matches_binding():
     n = w.workspace_bytes("full", p, 1, max_pages=16384)
     assert n > 0 and n % 256 == 0
     assert w.workspace_bytes("verify", p, 1, num_q=4, max_pages=16384) >= n
+
+
+def test_verify_flags_values_beyond_fp16_range():
+    """The verify value product runs in fp16; a V value of 2^16 or more must
+    raise the range bit instead of passing silently."""
+    p = _params(16, 2, 256, 64)
+    kv = _paged(95, 1, 2, 256, 64, [300])
+    kv.v_pool[kv.page_table[0, 1], 1, 5, 7] = 1.0e5
+    q = synth.queries(96, (1, 4, 16, 256), device=DEV)
+    status = w.new_status(DEV)
+    w.verify_attn(p, q, cache_of(kv), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & L.DEV_V_RANGE
