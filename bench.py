@@ -94,16 +94,45 @@ def barrier(world: int):
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and throttle reasons sampled every few milliseconds during the
+    timed region: NVML queries from a background thread (read-only), else
+    `nvidia-smi -lms`."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_S = 0.005
 
-    def __init__(self, device_index: int, enabled: bool = True):
+    def __init__(self, device_index, enabled: bool = True, uuid: str | None = None):
         self.proc = None
+        self.thread = None
         self.idx = device_index
         self.lines = []
+        self.samples = []
+        self.max_mhz = None
         if not enabled:
             return
+        try:
+            import threading
+
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            if uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+                except pynvml.NVMLError:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(device_index))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.nv = pynvml
+            self.handle = h
+            self.running = True
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # no NVML: fall back to nvidia-smi
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
@@ -111,7 +140,35 @@ class ClockSampler:
         except (OSError, ValueError):
             self.proc = None
 
+    def _poll(self):
+        nv, h = self.nv, self.handle
+        while self.running:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), int(reasons)))
+            except Exception:
+                pass
+            time.sleep(self.INTERVAL_S)
+
+    def _stop_nvml(self):
+        self.running = False
+        self.thread.join(timeout=5)
+        nv = self.nv
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+                "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown}
+        if not self.samples:
+            return None
+        reasons = sorted({name for _, r in self.samples for name, bit in bits.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
+
     def stop(self):
+        if self.thread is not None:
+            return self._stop_nvml()
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -137,7 +194,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -323,9 +380,10 @@ def algorithmic_bytes(wl, kind: str, ctx: int) -> float:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (baseline, not target)
 # ---------------------------------------------------------------------------
-def oracle_step_model(args, sample_ctx: int):
-    """Time the fp64 oracle on one sample of each unit at `sample_ctx` tokens,
-    return modelled microseconds per decode step at the workload's context."""
+def oracle_step_model(args, sample_ctx: int, repeats: int = 1):
+    """Time the fp64 oracle on one sample of each unit at `sample_ctx` tokens
+    (the fastest of `repeats` runs of each), return modelled microseconds per
+    decode step at the workload's context."""
     import numpy as np
 
     import oracle
@@ -345,12 +403,16 @@ def oracle_step_model(args, sample_ctx: int):
     q1 = synth.queries(7, (1, Hq, D)).double().numpy()
     qv = synth.queries(8, (1, gamma + 1, Hq, D)).double().numpy()
     scale = 1 / math.sqrt(D)
-    t0 = time.perf_counter()
-    oracle.draft_attn_full(q1, kp, vp, pt, np.array([n + 1]), P, scale)
-    t_draft = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    oracle.verify_attn(qv, kp, vp, pt, np.array([n + gamma + 1]), P, scale)
-    t_ver = time.perf_counter() - t0
+    t_draft = t_ver = math.inf
+    work = 0.0
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.draft_attn_full(q1, kp, vp, pt, np.array([n + 1]), P, scale)
+        t1 = time.perf_counter()
+        oracle.verify_attn(qv, kp, vp, pt, np.array([n + gamma + 1]), P, scale)
+        t2 = time.perf_counter()
+        t_draft, t_ver = min(t_draft, t1 - t0), min(t_ver, t2 - t1)
+        work += t2 - t0
     # windowed: the ring holds S+W entries whatever the context
     ring = oracle.RingModel(S, W, gamma, Hkv, D, dtype=np.float64)
     m = min(n, S + W)
@@ -363,7 +425,7 @@ def oracle_step_model(args, sample_ctx: int):
     f = ctx_full / n
     native_us = (gamma * t_draft * f + L * t_ver * f) * 1e6
     windowed_us = (gamma * t_win + L * t_ver * f) * 1e6
-    return {"native_us": native_us, "windowed_us": windowed_us, "sample_ctx": n, "work_s": t_draft + t_ver + t_win,
+    return {"native_us": native_us, "windowed_us": windowed_us, "sample_ctx": n, "work_s": work + t_win,
             "t_draft_s": t_draft, "t_verify_s": t_ver, "t_windowed_s": t_win}
 
 
@@ -376,6 +438,40 @@ def cores_used():
     except Exception:
         pass
     return len(os.sched_getaffinity(0))
+
+
+# DRAM traffic of one verify_tc_kernel launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from one ncu capture of this script on the default
+# workload.  It is reported as roofline.traffic only while the kernel source
+# hashes to the value it was captured on, and only for that workload.
+VERIFY_TRAFFIC = {
+    "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
+    "sha256": "5d18d149e0cd20b5bf28d978d2df50729636ad14861ca5e45080aa359b48416f",
+    "workload": "1m: batch 1, 16q/2kv heads, D=256, page 64, ctx 1048576, S=4, W=4096, gamma=3, 10 verify layers",
+    "bytes": 2.15e9 + 3.41e6,  # ncu prints three significant digits: 2.15 GB read, 3.41 MB written
+}
+
+
+def verify_traffic(desc: str):
+    import hashlib
+    if VERIFY_TRAFFIC["bytes"] is None or desc != VERIFY_TRAFFIC["workload"]:
+        return None
+    h = hashlib.sha256()
+    for rel in VERIFY_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return VERIFY_TRAFFIC["bytes"] if h.hexdigest() == VERIFY_TRAFFIC["sha256"] else None
+
+
+def workload_desc(args) -> str:
+    """The workload string of `config`, shared by both arms."""
+    import synth
+    base = synth.workload(args.config)
+    W = args.window if args.config in ("1m", "128k") else base.window
+    L = args.layers if args.layers is not None else base.verify_layers
+    return (f"{args.config}: batch {base.batch}, {base.num_heads_q}q/{base.num_heads_kv}kv heads, "
+            f"D={base.head_dim}, page {base.page_size}, ctx {base.context[0]}, S={base.sinks}, W={W}, "
+            f"gamma={args.gamma}, {L} verify layers")
 
 
 def run_reference(args):
@@ -396,7 +492,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "us/step", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.config, "gamma": args.gamma, "window": args.window, "sinks": 4,
+        "config": {"workload": workload_desc(args),
                    "native_us_per_step": statistics.median(x["native_us"] for x in per)},
         "cpu_baseline": {"value": v, "unit": "us/step", "cores": cores_used(), "kind": "oracle",
                          "sample": f"one native draft, one windowed draft and one verify layer at {sample} "
@@ -454,7 +550,11 @@ def main():
     # different ring, and neither reads the other's state
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     smi_id = vis.split(",")[torch.cuda.current_device()].strip() if vis else str(torch.cuda.current_device())
-    clocks = ClockSampler(smi_id, enabled=not args.no_clocks and rank == 0)
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except (AttributeError, RuntimeError):
+        uuid = None
+    clocks = ClockSampler(smi_id, enabled=not args.no_clocks and rank == 0, uuid=uuid)
     ms_win, ev_win = timed("windowed", True)
     ms_nat, ev_nat = timed("native", True)
     clk = clocks.stop()
@@ -525,11 +625,12 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = oracle_step_model(args, 262144)
+        r = oracle_step_model(args, 524288, repeats=2)
         cpu = {"value": r["windowed_us"], "unit": "us/step", "cores": cores_used(), "kind": "oracle",
                "sample": (f"fp64 numpy oracle: one native draft, one windowed draft and one verify layer at "
-                          f"{r['sample_ctx']} tokens (batch 1, 16/2 heads, D=256), scaled linearly in "
-                          f"context to {ctx}; {r['work_s']:.1f} s of CPU work"),
+                          f"{r['sample_ctx']} tokens (batch 1, 16/2 heads, D=256; draft and verify timed "
+                          f"twice, the faster kept), scaled linearly in context to {ctx}; "
+                          f"{r['work_s']:.1f} s of CPU work"),
                "native_value": r["native_us"]}
 
     if rank != 0:
@@ -549,8 +650,7 @@ def main():
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": f"{args.config}: batch {wk.B}, {wk.Hq}q/{wk.Hkv}kv heads, D={wk.D}, page {wk.P}, "
-                        f"ctx {ctx}, S={wk.S}, W={wk.W}, gamma={wk.gamma}, {wk.L} verify layers",
+            "workload": workload_desc(args),
             "l2": "inputs larger than L2 (verify reads ~2 GiB per layer per step); the ring stays L2-warm "
                   "between the draft steps of one decode step",
             "native_us_per_step": us_nat,
@@ -566,8 +666,10 @@ def main():
             "device_status": status,
         },
         "roofline": {"bound": "hbm", "achieved": ver_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": ver_gbs / hbm_peak, "traffic": None, "kernel": "verify (decode_attn + combine)",
-                     "peak_source": peak_src},
+                     "frac": ver_gbs / hbm_peak, "traffic": verify_traffic(workload_desc(args)),
+                     "kernel": "verify_tc_kernel: algorithmic bytes of one verify call / CUDA-event time of the "
+                               "call (verify_tc_kernel + its split-KV combine)",
+                     "algorithmic_bytes": ver_bytes, "peak_source": peak_src},
         "e2e": e2e,
         "gpu_launches": wk.launches_per_step("windowed") * args.steps,
         "clocks": clk,
