@@ -31,6 +31,7 @@ from .attention import (  # noqa: F401
     bf16_bits_to_f64,
     attend,
     attend_rows,
+    attend_prefixes,
     causal_positions,
     full_positions,
     gather_paged,

@@ -130,6 +130,40 @@ def attend_rows(qs: np.ndarray, keys: np.ndarray, values: np.ndarray, sm_scale: 
     return np.stack(outs), np.asarray(lses, dtype=np.float64)
 
 
+def attend_prefixes(qs: np.ndarray, keys: np.ndarray, values: np.ndarray, lengths, sm_scale: float):
+    """Row ``r`` of ``qs`` attends the first ``lengths[r]`` keys (fp64).
+
+    The ``attend`` definition for several queries whose key sets are prefixes
+    of one key list: a causal verify block (query ``i`` sees positions
+    ``0 .. n+i``) or draft steps at growing lengths.  One score matrix serves
+    every row; scores past a row's length are excluded before its maximum,
+    exponentials and sums are taken.  qs ``[R, D]``, keys/values ``[n, D]``,
+    lengths ``[R]`` with ``0 <= lengths[r] <= n`` -> (o ``[R, D]``, lse
+    ``[R]``); an empty prefix gives (0, -inf).
+    """
+    qs = np.asarray(qs, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    values = np.asarray(values, dtype=np.float64)
+    lengths = np.asarray(lengths, dtype=np.int64).reshape(-1)
+    R, D = qs.shape
+    n = keys.shape[0]
+    if lengths.shape[0] != R or (lengths < 0).any() or (lengths > n).any():
+        raise ValueError("need one length per row, each in [0, n]")
+    o = np.zeros((R, D), dtype=np.float64)
+    lse = np.full(R, EMPTY_LSE, dtype=np.float64)
+    live = lengths > 0
+    if n == 0 or not live.any():
+        return o, lse
+    s = float(sm_scale) * (keys @ qs.T)                          # [n, R]
+    s[np.arange(n)[:, None] >= lengths[None, :]] = -np.inf        # outside the prefix
+    m = np.where(live, s.max(axis=0), 0.0)
+    p = np.exp(s - m[None, :])                                    # exp(-inf) = 0
+    l = p.sum(axis=0)
+    o[live] = (p.T @ values)[live] / l[live, None]
+    lse[live] = m[live] + np.log(l[live])
+    return o, lse
+
+
 def gather_paged(pool: np.ndarray, table_row: np.ndarray, positions: np.ndarray,
                  page_size: int, kv_head: int) -> np.ndarray:
     """Rows of one KV head at ``positions`` from a ``[pages, Hkv, P, D]`` pool."""

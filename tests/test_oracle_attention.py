@@ -149,6 +149,42 @@ def test_attend_permutation_invariance_and_empty():
     assert np.all(o == 0) and lse == -np.inf
 
 
+def test_attend_prefixes_matches_torch_sdpa_with_prefix_mask():
+    # library pin: float64 SDPA with a boolean mask that keeps key t for row r
+    # iff t < lengths[r] (the causal-verify and growing-draft shapes)
+    r = _rng(11)
+    n, d, R = 37, 16, 6
+    K, V, Q = r.standard_normal((n, d)), r.standard_normal((n, d)), r.standard_normal((R, d))
+    lengths = np.array([1, 5, 36, 37, 20, 2])
+    o, lse = A.attend_prefixes(Q, K, V, lengths, 0.3)
+    mask = np.arange(n)[None, :] < lengths[:, None]
+    np.testing.assert_allclose(o, _sdpa(Q, K, V, 0.3, mask), atol=1e-12, rtol=0)
+    s = 0.3 * (Q @ K.T)
+    ref_lse = torch.logsumexp(torch.from_numpy(np.where(mask, s, -np.inf)), -1).numpy()
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-12, rtol=0)
+
+
+def test_attend_prefixes_bruteforce_and_edges():
+    # pure-Python loops on a tiny case, an empty prefix, and the full prefix
+    r = _rng(12)
+    n, d = 6, 3
+    K, V, Q = r.standard_normal((n, d)), r.standard_normal((n, d)), r.standard_normal((3, d))
+    lengths = [0, 4, 6]
+    o, lse = A.attend_prefixes(Q, K, V, lengths, 0.5)
+    assert np.all(o[0] == 0) and lse[0] == -np.inf
+    for row in (1, 2):
+        L_ = lengths[row]
+        sc = [0.5 * sum(Q[row, c] * K[t, c] for c in range(d)) for t in range(L_)]
+        mx = max(sc)
+        ex = [math.exp(x - mx) for x in sc]
+        tot = sum(ex)
+        for c in range(d):
+            assert abs(o[row, c] - sum(ex[t] * V[t, c] for t in range(L_)) / tot) < 1e-12
+        assert abs(lse[row] - (mx + math.log(tot))) < 1e-12
+    with pytest.raises(ValueError):
+        A.attend_prefixes(Q, K, V, [1, 2, 7], 0.5)
+
+
 def test_bf16_widening_is_exact():
     x = torch.randn(1000, dtype=torch.float32).to(torch.bfloat16)
     bits = x.view(torch.int16).numpy().view(np.uint16)
@@ -343,6 +379,6 @@ def test_combine_all_empty_and_matches_torch_logsumexp():
 
 
 def test_oracle_package_exports():
-    for name in ["attend", "draft_attn_full", "draft_attn_windowed", "verify_attn",
+    for name in ["attend", "attend_prefixes", "draft_attn_full", "draft_attn_windowed", "verify_attn",
                  "splitkv_combine", "RingModel", "window_positions"]:
         assert hasattr(oracle, name)
