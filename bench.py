@@ -51,6 +51,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the steps as eager launches instead of one CUDA graph per decode step")
     return ap.parse_args(argv)
 
 
@@ -312,9 +314,11 @@ class Workload:
         return self.gamma * (1 + 2) + self.L * (1 + 2)
 
     # -- one decode step; `ev` collects (kind, start_event, end_event)
-    def step(self, s: int, arm: str, ev=None, inputs=None):
+    def step(self, s: int, arm: str, ev=None, inputs=None, external_events: bool = False):
         torch, w = self.torch, self.w
-        E = torch.cuda.Event
+
+        def E(**kw):  # events inside a captured graph must be graph nodes
+            return torch.cuda.Event(external=external_events, **kw)
         qd = self.q_draft[s] if inputs is None else inputs["q_draft"]
         qv = self.q_ver[s] if inputs is None else inputs["q_ver"]
         for j in range(self.gamma):
@@ -537,6 +541,20 @@ def main():
     if int(wk.status.item()) != 0:
         raise SystemExit(f"device status {int(wk.status.item()):#x} during warmup")
 
+    # One CUDA graph per timed decode step and arm (the step's ~40 library
+    # launches replay without host gaps); --eager launches them from Python.
+    graphs = {}
+    if not args.eager:
+        for arm in ("windowed", "native"):
+            graphs[arm] = []
+            for s in range(args.warmup, args.warmup + args.steps):
+                evs = []
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    wk.step(s, arm, ev=evs, external_events=True)
+                graphs[arm].append((g, evs))
+        torch.cuda.synchronize()
+
     def timed(arm, with_events):
         evs = [] if with_events else None
         wk.restore_ring(ring_after_warmup)
@@ -545,8 +563,14 @@ def main():
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         start.record()
-        for s in range(args.warmup, args.warmup + args.steps):
-            wk.step(s, arm, ev=evs)
+        if graphs:
+            for g, gev in graphs[arm]:
+                g.replay()
+                if evs is not None:
+                    evs.extend(gev)
+        else:
+            for s in range(args.warmup, args.warmup + args.steps):
+                wk.step(s, arm, ev=evs)
         end.record()
         torch.cuda.synchronize()
         barrier(world)
@@ -660,6 +684,7 @@ def main():
             "workload": workload_desc(args),
             "l2": "inputs larger than L2 (verify reads ~2 GiB per layer per step); the ring stays L2-warm "
                   "between the draft steps of one decode step",
+            "launch": "eager Python launches" if args.eager else "one CUDA graph per decode step and arm",
             "native_us_per_step": us_nat,
             "windowed_us_per_step": us_win,
             "native_over_windowed": us_nat / us_win,

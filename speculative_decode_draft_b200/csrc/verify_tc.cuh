@@ -70,7 +70,7 @@ struct TcPlan {
   static constexpr int kOffBar = STAGES * kStageBytes;
   // k_full[S], k_empty[S], v_full[S], v_empty[S], v_ready[S], s_full[2],
   // p_full[2], o_done, mma_final
-  static constexpr int kNumBars = 5 * STAGES + 6;
+  static constexpr int kNumBars = 5 * STAGES + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort
   static constexpr int kBytes = kOffMisc + 8;
   static constexpr int kAlloc = kBytes + 1024;
@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_o_done = bar_p_full + 16;
   const uint32_t bar_final = bar_o_done + 8;
+  const uint32_t bar_q_ready = bar_final + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
 
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     ptx::mbar_init(bar_o_done, 1);
     ptx::mbar_init(bar_final, 1);
+    ptx::mbar_init(bar_q_ready, 4);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -164,29 +166,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const bool row_active = warp >= 2 && warp < 6 && lane < 16 && row < a.rows;
   const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
 
-  if (warp >= 2 && warp < 6) {
-    // Q row into TMEM columns 0..127 (bf16 pairs), zeros for padding rows
-    const __nv_bfloat16* src =
-        row_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
-                   : nullptr;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t w[32];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row_active) v = *reinterpret_cast<const uint4*>(src + 64 * c + 8 * j);
-        w[4 * j] = v.x;
-        w[4 * j + 1] = v.y;
-        w[4 * j + 2] = v.z;
-        w[4 * j + 3] = v.w;
-      }
-      tc::tmem_st32(tmem_base + lane_addr + kColQ + 32 * c, w);
-    }
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // =================================================================== producers
@@ -306,7 +285,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::commit(bar_s_full + 8 * (k & 1));
         tc::commit(bar_k_empty + 8 * (k % STAGES));
       };
-      bool ok = tc_wait(bar_k_full, 0, abort_flag);
+      // Q is staged into TMEM by the softmax warps while the first K/V tiles
+      // are in flight
+      bool ok = tc_wait(bar_q_ready, 0, abort_flag) && tc_wait(bar_k_full, 0, abort_flag);
       if (ok) {
         tc::fence_after_sync();
         issue_qk(0);
@@ -346,6 +327,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ================================================================= softmax
+    {
+      // Q row into TMEM columns 0..127 (bf16 pairs), zeros for padding rows;
+      // every load is issued before the first store so the row costs one
+      // global-memory round trip
+      const __nv_bfloat16* src =
+          row_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
+                     : nullptr;
+      uint4 v[D / 8];
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j)
+        v[j] = row_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t wq[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          wq[4 * j] = v[8 * c + j].x;
+          wq[4 * j + 1] = v[8 * c + j].y;
+          wq[4 * j + 2] = v[8 * c + j].z;
+          wq[4 * j + 3] = v[8 * c + j].w;
+        }
+        tc::tmem_st32(tmem_base + lane_addr + kColQ + 32 * c, wq);
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_q_ready);
+    }
     const int lim = row_active ? n_tok - a.num_q + row / a.G + 1 : n_tok;  // causal limit of this row
     const int first_masked_tok = n_tok - a.num_q + 1;
     float m_ref = -INFINITY;  // reference maximum (log2 units)
