@@ -150,6 +150,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // barriers first: with a programmatic launch this overlaps the previous
+  // kernel's tail; every global-memory access comes after griddepcontrol.wait
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(bar_full + 8 * s, 1);
+      ptx::mbar_init(bar_empty + 8 * s, kComputeWarps);
+    }
+    ptx::fence_mbar_init();
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // ---- the token range of this split (uniform across the CTA)
   int n_tok = 0;
   int seq_len = 0;
@@ -173,14 +184,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_begin = min(split * tps, ntiles);
   const int t_end = min(t_begin + tps, ntiles);
   const int my_tiles = t_end - t_begin;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(bar_full + 8 * s, 1);
-      ptx::mbar_init(bar_empty + 8 * s, kComputeWarps);
-    }
-    ptx::fence_mbar_init();
-  }
   __syncthreads();
   // let the dependent combine kernel get scheduled while this grid runs; it
   // waits in-kernel until this grid has finished and its writes are visible
@@ -195,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int box_rows = RING ? kTileTokens : min(a.page_size, kTileTokens);
       const int boxes = kTileTokens / box_rows;
       const int oob_z = RING ? 0x7fffffff : a.num_pages * a.Hkv;  // past the tensor: zero fill
+      int issued = 0;
       for (int k = 0; k < my_tiles; ++k) {
         const int stage = k % STAGES;
         const uint32_t par = ((k / STAGES) & 1) ^ 1;
@@ -252,7 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        issued = k + 1;
       }
+      // no copy may still be writing shared memory when the CTA exits (after
+      // a timeout the consumers stop early): wait, bounded, for the last load
+      // of each stage
+      for (int k = max(issued - STAGES, 0); k < issued; ++k)
+        if (!ptx::mbar_wait(bar_full + 8 * (k % STAGES), (k / STAGES) & 1)) set_status(a.status, kDevTimeout);
     }
     return;
   }

@@ -6,23 +6,25 @@
 // share each K/V byte; with G = 8 that is 16..64 rows against every token.
 //
 // Per CTA = (split, KV head, sequence), head_dim 256, 64-token tiles, with
-// the rows as the MMA M dimension (padded to 128) and everything but K and V
-// kept in tensor memory (512 columns x 128 lanes):
+// the rows as the MMA M dimension (padded to 64) and everything but K and V
+// kept in tensor memory (512 columns; the M=64 layout uses lanes 0..15 of
+// each of the four lane quadrants):
 //   columns   0..127  Q            bf16 pairs, the A operand of S = Q K^T
 //   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax
 //                                  columns 0..31 of the buffer hold P as fp16
 //                                  pairs, the A operand of P V
 //   columns 256..511  O            fp32 output accumulator, 256 head dims
-// Row r of the block sits in TMEM lane 32 (r % 4) + r / 4, so the rows spread
-// over the four lane quadrants and each softmax warp owns a quarter of them.
+// Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
+// 16 (r % 4) + r / 4), so the rows spread over the four lane quadrants and
+// each softmax warp owns a quarter of them.
 //
 // Roles: warp 0 streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
 // into two STAGES-deep shared-memory rings with TMA, one lane per ring: a K
 // tile is released as soon as its S = Q K^T has completed, a V tile only
 // after its O += P V, so K loads run ahead of the softmax instead of waiting
 // for the slower PV of the same tile; warp 1 allocates the tensor
-// memory and one lane issues every MMA (S = Q K^T as M=128, N=64 with K from
-// shared memory, K-major; O += P V as M=128, N=256 with V read MN-major
+// memory and one lane issues every MMA (S = Q K^T as M=64, N=64 with K from
+// shared memory, K-major; O += P V as M=64, N=256 with V read MN-major
 // straight from the TMA tile); warps 2..5 run the softmax, one thread per
 // row: the row's scores come out of TMEM, the maximum and sum are taken
 // inside the thread, and P goes back into TMEM in fp16; warps 6..9 convert
@@ -120,18 +122,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- token range of this split
-  int n_tok = a.kv_len[b];
-  if (n_tok != 0 && (n_tok < a.num_q || n_tok > a.max_pages * a.page_size)) {
-    if (threadIdx.x == 0 && split == 0 && kvh == 0) set_status(a.status, kDevLenOob);
-    n_tok = 0;
-  }
-  const int ntiles = (n_tok + kTileTokens - 1) / kTileTokens;
-  const int tps = (ntiles + a.nsplit - 1) / a.nsplit;
-  const int t_begin = min(split * tps, ntiles);
-  const int t_end = min(t_begin + tps, ntiles);
-  const int my_tiles = t_end - t_begin;
-
   // ---- set-up: barriers and tensor memory
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -155,6 +145,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
     tc::tmem_relinquish();
   }
+  // every global-memory access comes after this: with a programmatic launch
+  // the set-up above overlaps the previous kernel's tail
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- token range of this split
+  int n_tok = a.kv_len[b];
+  if (n_tok != 0 && (n_tok < a.num_q || n_tok > a.max_pages * a.page_size)) {
+    if (threadIdx.x == 0 && split == 0 && kvh == 0) set_status(a.status, kDevLenOob);
+    n_tok = 0;
+  }
+  const int ntiles = (n_tok + kTileTokens - 1) / kTileTokens;
+  const int tps = (ntiles + a.nsplit - 1) / a.nsplit;
+  const int t_begin = min(split * tps, ntiles);
+  const int t_end = min(t_begin + tps, ntiles);
+  const int my_tiles = t_end - t_begin;
+  // start the page-table reads of the first tiles now; the producers' own
+  // loads then hit L2
+  if (warp == 0 && lane < STAGES && lane < my_tiles) {
+    const int* pte = a.page_table + static_cast<size_t>(b) * a.max_pages +
+                     ((t_begin + lane) * kTileTokens) / a.page_size;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(pte));
+  }
+
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -182,6 +195,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
       const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
       const uint32_t ring = sbase + Plan::kOffK + (is_k ? 0 : Plan::kTileBytes);
+      int issued = 0;
       for (int k = 0; k < my_tiles; ++k) {
         const int stage = k % STAGES;
         if (!tc_wait(bar_empty + 8 * stage, ((k / STAGES) & 1) ^ 1, abort_flag)) {
@@ -215,7 +229,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < 4; ++c)
             ptx::tma_load_3d(dst + c * Plan::kChunkBytes + j * box_rows * 128, tmap, fb, c * 64, ys[j], zs[j], pol);
         }
+        issued = k + 1;
       }
+      // no copy may still be writing shared memory when the CTA exits (after
+      // an abort the consumers stop early): wait, bounded, for the last load
+      // of each stage
+      for (int k = max(issued - STAGES, 0); k < issued; ++k)
+        if (!ptx::mbar_wait(bar_full + 8 * (k % STAGES), (k / STAGES) & 1)) set_status(a.status, kDevTimeout);
     }
     return;
   }
@@ -268,8 +288,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // =================================================================== MMA issuer
   if (warp == 1) {
     if (lane == 0 && my_tiles > 0) {
-      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(128, 64, 0, 0);   // A (Q, TMEM), B (K) K-major
-      constexpr uint32_t kIdescPV = tc::idesc_f16_f32(128, 256, 0, 1);   // A (P, TMEM), B (V) MN-major, fp16
+      // M = 64: the rows never exceed 64, and an M=64 MMA costs the same
+      // issue time as M=128 for half the tensor work (and power)
+      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(64, 64, 0, 0);    // A (Q, TMEM), B (K) K-major
+      constexpr uint32_t kIdescPV = tc::idesc_f16_f32(64, 256, 0, 1);    // A (P, TMEM), B (V) MN-major, fp16
       // descriptor start addresses are in 16-byte units in the low bits, so
       // moving an operand by n bytes adds n >> 4 to the descriptor
       const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
@@ -450,17 +472,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     // ---- finish: normalised partial output and log-sum-exp of this row
     if (!failed && my_tiles > 0) {
-      // o_done completes once per PV.  When the last S arrived, PV(n-3) had
-      // completed (it was issued before that QK) but PV(n-2) may not have, so
-      // wait for the phases of PV(n-2) and PV(n-1) in turn: a parity wait
-      // only tells the pending phase from the one just before it.
-      bool done = true;
-      if (my_tiles >= 2) done = tc_wait(bar_o_done, (my_tiles - 2) & 1, abort_flag);
-      done = done && tc_wait(bar_o_done, (my_tiles - 1) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, done)) failed = true;
+      // mma_final completes once, when every MMA of the CTA has completed (a
+      // parity wait on o_done could not tell PV(n-2)'s phase from PV(n)'s
+      // once both PV(n-2) and PV(n-1) have completed)
+      if (!__all_sync(0xffffffffu, tc_wait(bar_final, 0, abort_flag))) failed = true;
       tc::fence_after_sync();
     }
-    failed = __any_sync(0xffffffffu, failed);
+    failed = __any_sync(0xffffffffu, failed || *abort_flag != 0);
     if (failed) {
       if (lane == 0) set_status(a.status, kDevTimeout);
       *abort_flag = 1;
@@ -470,18 +488,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         row_active ? (static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G : 0;
     float* dst = a.part_o + (grow * a.nsplit + split) * D;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      uint32_t o[32];
+    for (int c = 0; c < 2; ++c) {  // two 128-column TMEM loads per row
+      uint32_t o[128];
       if (my_tiles > 0 && !failed) {
-        tc::tmem_ld32(tmem_base + lane_addr + kColO + 32 * c, o);
+        tc::tmem_ld128(tmem_base + lane_addr + kColO + 128 * c, o);
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = 0u;
+        for (int j = 0; j < 128; ++j) o[j] = 0u;
       }
       if (row_active) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + 32 * c + j) =
+        for (int j = 0; j < 128; j += 4)
+          *reinterpret_cast<float4*>(dst + 128 * c + j) =
               make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
                           __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
       }

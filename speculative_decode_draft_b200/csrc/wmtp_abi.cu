@@ -145,6 +145,27 @@ LaunchPlan make_plan(int sms, int B, int Hkv, long long rows_total, int D, int N
   return pl;
 }
 
+// Launch an attention kernel as a programmatic dependent of whatever the
+// stream ran before: its barrier and tensor-memory set-up may overlap that
+// kernel's tail, and it executes griddepcontrol.wait before its first
+// global-memory access, so stream order is kept for every byte it reads.
+template <typename Kern>
+wmtp_status launch_programmatic(Kern kern, dim3 grid, int threads, int smem, cudaStream_t st,
+                                const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tk, tv, a) == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- dispatch
 template <int D, int NT, bool RING>
 wmtp_status launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
@@ -161,9 +182,7 @@ wmtp_status launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const 
       return WMTP_ERR_CUDA;
     attr_done[dev] = true;
   }
-  dim3 grid(a.nsplit, a.Hkv, B);
-  kern<<<grid, kThreads, alloc, st>>>(tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  return launch_programmatic(kern, dim3(a.nsplit, a.Hkv, B), kThreads, alloc, st, tk, tv, a);
 }
 
 template <bool RING>
@@ -193,9 +212,7 @@ wmtp_status launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const
       return WMTP_ERR_CUDA;
     attr_done[dev] = true;
   }
-  dim3 grid(a.nsplit, a.Hkv, B);
-  kern<<<grid, kTcThreads, alloc, st>>>(tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  return launch_programmatic(kern, dim3(a.nsplit, a.Hkv, B), kTcThreads, alloc, st, tk, tv, a);
 }
 
 // Verify blocks of head_dim 256 with 9..64 query rows run on tcgen05.
