@@ -55,6 +55,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--ctx", type=int, default=None, help="committed context length (default: the config's)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="context x gamma x window sweep of native/windowed step time (one JSON line per point)")
     ap.add_argument("--eager", action="store_true",
                     help="time the steps as eager launches instead of one CUDA graph per decode step")
     return ap.parse_args(argv)
@@ -236,7 +239,7 @@ class Workload:
         self.gamma = args.gamma
         self.L = args.layers if args.layers is not None else base.verify_layers
         self.steps_total = args.steps + args.warmup
-        self.n0 = base.context[0]
+        self.n0 = args.ctx if args.ctx else base.context[0]
         seed = base.seed + 1000 * rank
         self.seed = seed
         dev = device
@@ -485,8 +488,9 @@ def workload_desc(args) -> str:
     base = synth.workload(args.config)
     W = args.window if args.config in ("1m", "128k") else base.window
     L = args.layers if args.layers is not None else base.verify_layers
+    ctx = args.ctx if args.ctx else base.context[0]
     return (f"{args.config}: batch {base.batch}, {base.num_heads_q}q/{base.num_heads_kv}kv heads, "
-            f"D={base.head_dim}, page {base.page_size}, ctx {base.context[0]}, S={base.sinks}, W={W}, "
+            f"D={base.head_dim}, page {base.page_size}, ctx {ctx}, S={base.sinks}, W={W}, "
             f"gamma={args.gamma}, {L} verify layers")
 
 
@@ -519,24 +523,12 @@ def run_reference(args):
     return 0
 
 
-# ---------------------------------------------------------------------------
-def main():
-    args = parse()
-    if args.impl == "reference":
-        return run_reference(args)
+def time_arms(args, wk, world: int, make_clocks=None) -> dict:
+    """Warm up both arms, capture each timed step as a CUDA graph (unless
+    --eager), then time K steps of each arm, windowed and native alternating,
+    between a barrier + synchronize on both sides.  Returns per-arm device ms
+    (max over ranks), per-call means by kind (us) and the clock record."""
     import torch
-
-    import speculative_decode_draft_b200 as w
-    from speculative_decode_draft_b200 import build
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    rank, world, local = dist_setup(args)
-    build.build()
-    w.load()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    wk = Workload(args, rank, dev)
-    stream = torch.cuda.current_stream()
-
     # ---------------- warmup (both arms)
     for s in range(args.warmup):
         wk.step(s, "native")
@@ -589,15 +581,9 @@ def main():
 
     # the windowed arm advances the ring; the native arm must not see a
     # different ring, and neither reads the other's state
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    smi_id = vis.split(",")[torch.cuda.current_device()].strip() if vis else str(torch.cuda.current_device())
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    except (AttributeError, RuntimeError):
-        uuid = None
-    clocks = ClockSampler(smi_id, enabled=not args.no_clocks and rank == 0, uuid=uuid)
+    clocks = make_clocks() if make_clocks else None
     ms_arm, ev_arm = timed_interleaved()
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     ms_win = max_over_ranks(ms_arm["windowed"], world)
     ms_nat = max_over_ranks(ms_arm["native"], world)
     ev_win, ev_nat = ev_arm["windowed"], ev_arm["native"]
@@ -608,8 +594,70 @@ def main():
             out.setdefault(kind, []).append(a.elapsed_time(b) * 1000.0)
         return {k: statistics.mean(v) for k, v in out.items()}
 
-    k_win = per_kind(ev_win)
-    k_nat = per_kind(ev_nat)
+    return {"ms_win": ms_win, "ms_nat": ms_nat, "k_win": per_kind(ev_win), "k_nat": per_kind(ev_nat),
+            "clocks": clk, "ring_after_warmup": ring_after_warmup}
+
+
+def run_sweep(args, rank: int, world: int, dev) -> int:
+    """The pages' windowing wedge, step^native / step^windowed - 1, over
+    context, draft depth and window (one JSON line per point, rank 0)."""
+    import copy
+
+    import torch
+    contexts = (2048, 8192, 32768, 131072, 524288, 1048576)
+    points = [(c, g, 2048) for c in contexts for g in (1, 3, 5, 7)]
+    points += [(c, 3, W) for c in contexts for W in (1024, 4096, 8192)]
+    for ctx, gamma, window in points:
+        a = copy.copy(args)
+        a.config, a.ctx, a.gamma, a.window = "1m", ctx, gamma, window
+        wk = Workload(a, rank, dev)
+        r = time_arms(a, wk, world)
+        if int(wk.status.item()) != 0:
+            raise SystemExit(f"device status {int(wk.status.item()):#x} at ctx {ctx} gamma {gamma} W {window}")
+        win = whole_job_us_per_step(r["ms_win"], a.steps, world)
+        nat = whole_job_us_per_step(r["ms_nat"], a.steps, world)
+        if rank == 0:
+            print(json.dumps({"sweep": True, "ctx": ctx, "gamma": gamma, "window": window, "layers": wk.L,
+                              "windowed_us": win, "native_us": nat, "wedge": nat / win - 1.0,
+                              "bytes_implied_wedge": gamma * (1.0 - min(ctx, 4 + window) / ctx) / wk.L,
+                              "draft_windowed_us": r["k_win"]["draft"], "draft_native_us": r["k_nat"]["draft"],
+                              "verify_us": r["k_win"]["verify"]}), flush=True)
+        del wk, r
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+
+    import speculative_decode_draft_b200 as w
+    from speculative_decode_draft_b200 import build
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    rank, world, local = dist_setup(args)
+    build.build()
+    w.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if args.sweep:
+        return run_sweep(args, rank, world, dev)
+    wk = Workload(args, rank, dev)
+    stream = torch.cuda.current_stream()
+
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except (AttributeError, RuntimeError):
+        uuid = None
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[torch.cuda.current_device()].strip() if vis else str(torch.cuda.current_device())
+    r = time_arms(args, wk, world,
+                  lambda: ClockSampler(smi_id, enabled=not args.no_clocks and rank == 0, uuid=uuid))
+    ms_win, ms_nat, k_win, k_nat, clk = r["ms_win"], r["ms_nat"], r["k_win"], r["k_nat"], r["clocks"]
+    ring_after_warmup = r["ring_after_warmup"]
     ctx = wk.n0
     peaks = {}
     try:
