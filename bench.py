@@ -48,7 +48,7 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["wmtp", "reference"], default="wmtp")
-    ap.add_argument("--config", default="1m", choices=["tiny", "32k", "128k", "1m"])
+    ap.add_argument("--config", default="1m", choices=["tiny", "32k", "128k", "1m", "ragged4"])
     ap.add_argument("--gamma", type=int, default=3)
     ap.add_argument("--window", type=int, default=4096)
     ap.add_argument("--layers", type=int, default=None, help="verify layers (default: workload's)")
@@ -239,7 +239,9 @@ class Workload:
         self.gamma = args.gamma
         self.L = args.layers if args.layers is not None else base.verify_layers
         self.steps_total = args.steps + args.warmup
-        self.n0 = args.ctx if args.ctx else base.context[0]
+        # committed context per sequence at the first step (ragged4: one per sequence)
+        self.n0s = [int(args.ctx)] * base.batch if args.ctx else [int(c) for c in base.context]
+        self.n0 = max(self.n0s)
         seed = base.seed + 1000 * rank
         self.seed = seed
         dev = device
@@ -248,7 +250,7 @@ class Workload:
         self.accept = synth.accept_counts(seed, self.steps_total, self.B, self.gamma)
         # committed length at the start of each step
         self.n_at = np.zeros((self.steps_total + 1, self.B), dtype=np.int64)
-        self.n_at[0] = self.n0
+        self.n_at[0] = self.n0s
         for s in range(self.steps_total):
             self.n_at[s + 1] = self.n_at[s] + self.accept[s]
         cap = int(self.n_at[-1].max()) + self.gamma + 2 + self.P
@@ -257,10 +259,10 @@ class Workload:
         kvs = base.kv_scale
         shuf = base.shuffle_pages
         # verify layers: independent random KV, n0 committed tokens each
-        self.layers = [synth.paged_kv(seed + 10 + l, self.B, self.Hkv, self.D, self.P, [self.n0] * self.B,
+        self.layers = [synth.paged_kv(seed + 10 + l, self.B, self.Hkv, self.D, self.P, self.n0s,
                                       cap, kvs, shuf, device=dev) for l in range(self.L)]
         # the draft layer's own KV (native arm reads it in full)
-        self.draft = synth.paged_kv(seed + 5, self.B, self.Hkv, self.D, self.P, [self.n0] * self.B, cap, kvs,
+        self.draft = synth.paged_kv(seed + 5, self.B, self.Hkv, self.D, self.P, self.n0s, cap, kvs,
                                     shuf, device=dev)
         self.caches = [w.PagedCache(k.k_pool, k.v_pool, k.page_table, k.kv_len) for k in self.layers]
         self.draft_cache = w.PagedCache(self.draft.k_pool, self.draft.v_pool, self.draft.page_table,
@@ -300,13 +302,13 @@ class Workload:
         self.l_ver = torch.empty(self.B, self.gamma + 1, self.Hq, **f32)
         # ring of the windowed arm, filled from the draft layer's history
         self.ring = w.Ring.allocate(self.p, self.B, dev)
-        kd = torch.empty(self.B, self.n0, self.Hkv, self.D, dtype=torch.bfloat16, device=dev)
-        vd = torch.empty_like(kd)
+        kd = torch.zeros(self.B, self.n0, self.Hkv, self.D, dtype=torch.bfloat16, device=dev)
+        vd = torch.zeros_like(kd)
         for b in range(self.B):
-            k, v = synth.dense_from_paged(self.draft, b, self.n0)
-            kd[b].copy_(k)
-            vd[b].copy_(v)
-        w.ring_append(self.p, self.ring, kd, vd, torch.full((self.B,), self.n0, **i32), status=self.status)
+            k, v = synth.dense_from_paged(self.draft, b, self.n0s[b])
+            kd[b, :self.n0s[b]].copy_(k)
+            vd[b, :self.n0s[b]].copy_(v)
+        w.ring_append(self.p, self.ring, kd, vd, torch.tensor(self.n0s, **i32), status=self.status)
         del kd, vd
         torch.cuda.synchronize()
         self.workspace = torch.empty(max(
@@ -381,18 +383,21 @@ class Workload:
             dst.copy_(src)
 
 
-def algorithmic_bytes(wl, kind: str, ctx: int) -> float:
-    """Bytes a call must move at context ctx (K and V of every attended token
-    for every KV head, plus queries, page-table entries and fp32 outputs)."""
+def algorithmic_bytes(wl, kind: str, ctxs) -> float:
+    """Bytes a call must move with committed contexts `ctxs` (one per
+    sequence): K and V of every attended token for every KV head, plus
+    queries, page-table entries and fp32 outputs."""
     kvb = 2 * wl.Hkv * wl.D * 2
     qn = wl.gamma + 1 if kind == "verify" else 1
-    q_bytes = wl.B * qn * wl.Hq * wl.D * 2
-    o_bytes = wl.B * qn * wl.Hq * (wl.D + 1) * 4
-    if kind == "windowed":
-        n_att = min(ctx, wl.S + wl.W)
-        return wl.B * n_att * (kvb + 4) + q_bytes + o_bytes
-    pt = math.ceil(ctx / wl.P) * 4
-    return wl.B * (ctx * kvb + pt) + q_bytes + o_bytes
+    q_bytes = len(ctxs) * qn * wl.Hq * wl.D * 2
+    o_bytes = len(ctxs) * qn * wl.Hq * (wl.D + 1) * 4
+    total = q_bytes + o_bytes
+    for ctx in ctxs:
+        if kind == "windowed":
+            total += min(ctx, wl.S + wl.W) * (kvb + 4)
+        else:
+            total += ctx * kvb + math.ceil(ctx / wl.P) * 4
+    return total
 
 
 # ---------------------------------------------------------------------------
@@ -411,8 +416,8 @@ def oracle_step_model(args, sample_ctx: int, repeats: int = 1):
     W = args.window if args.config in ("1m", "128k") else base.window
     gamma = args.gamma
     L = args.layers if args.layers is not None else base.verify_layers
-    ctx_full = base.context[0]
-    n = min(sample_ctx, ctx_full)
+    ctxs = [int(args.ctx)] * base.batch if args.ctx else [int(c) for c in base.context]
+    n = min(sample_ctx, max(ctxs))
     kv = synth.paged_kv(base.seed, 1, Hkv, D, P, [n + gamma + 1], n + gamma + 1 + P, base.kv_scale,
                         base.shuffle_pages, device="cpu")
     kp = kv.k_pool.double().numpy()
@@ -440,9 +445,9 @@ def oracle_step_model(args, sample_ctx: int, repeats: int = 1):
     t0 = time.perf_counter()
     oracle.draft_attn_windowed(q1, [ring], scale)
     t_win = time.perf_counter() - t0
-    f = ctx_full / n
+    f = sum(ctxs) / n  # every sequence's attention scales with its own context
     native_us = (gamma * t_draft * f + L * t_ver * f) * 1e6
-    windowed_us = (gamma * t_win + L * t_ver * f) * 1e6
+    windowed_us = (gamma * t_win * len(ctxs) + L * t_ver * f) * 1e6
     return {"native_us": native_us, "windowed_us": windowed_us, "sample_ctx": n, "work_s": work + t_win,
             "t_draft_s": t_draft, "t_verify_s": t_ver, "t_windowed_s": t_win}
 
@@ -488,7 +493,7 @@ def workload_desc(args) -> str:
     base = synth.workload(args.config)
     W = args.window if args.config in ("1m", "128k") else base.window
     L = args.layers if args.layers is not None else base.verify_layers
-    ctx = args.ctx if args.ctx else base.context[0]
+    ctx = args.ctx if args.ctx else "/".join(str(c) for c in base.context)
     return (f"{args.config}: batch {base.batch}, {base.num_heads_q}q/{base.num_heads_kv}kv heads, "
             f"D={base.head_dim}, page {base.page_size}, ctx {ctx}, S={base.sinks}, W={W}, "
             f"gamma={args.gamma}, {L} verify layers")
@@ -669,9 +674,9 @@ def main():
 
     class WL:  # shapes for the byte model
         B, Hq, Hkv, D, P, S, W, gamma = wk.B, wk.Hq, wk.Hkv, wk.D, wk.P, wk.S, wk.W, wk.gamma
-    ver_bytes = algorithmic_bytes(WL, "verify", ctx)
-    nat_bytes = algorithmic_bytes(WL, "full", ctx)
-    win_bytes = algorithmic_bytes(WL, "windowed", ctx)
+    ver_bytes = algorithmic_bytes(WL, "verify", wk.n0s)
+    nat_bytes = algorithmic_bytes(WL, "full", wk.n0s)
+    win_bytes = algorithmic_bytes(WL, "windowed", wk.n0s)
     ver_gbs = ver_bytes / (k_win["verify"] * 1e-6) / 1e9
     nat_gbs = nat_bytes / (k_nat["draft"] * 1e-6) / 1e9
     win_gbs = win_bytes / (k_win["draft"] * 1e-6) / 1e9
@@ -712,13 +717,30 @@ def main():
     torch.cuda.synchronize()
     status = int(wk.status.item())
 
+    # a read-only streaming reference (torch's sum over 4 GiB; context for the
+    # GB/s figures, not a peak the roofline divides by)
+    read_gbs = None
+    if not args.sweep:
+        big = torch.ones(1 << 31, dtype=torch.bfloat16, device=dev)
+        best = math.inf
+        for _ in range(4):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            big.sum(dtype=torch.float32)
+            a1.record()
+            torch.cuda.synchronize()
+            best = min(best, a0.elapsed_time(a1))
+        read_gbs = big.numel() * 2 / (best * 1e-3) / 1e9
+        del big
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_step_model(args, 524288, repeats=2)
         cpu = {"value": r["windowed_us"], "unit": "us/step", "cores": cores_used(), "kind": "oracle",
                "sample": (f"fp64 numpy oracle: one native draft, one windowed draft and one verify layer at "
                           f"{r['sample_ctx']} tokens (batch 1, 16/2 heads, D=256; draft and verify timed "
-                          f"twice, the faster kept), scaled linearly in context to {ctx}; "
+                          f"twice, the faster kept), scaled linearly in context to "
+                          f"{'/'.join(str(c) for c in wk.n0s)} tokens; "
                           f"{r['work_s']:.1f} s of CPU work"),
                "native_value": r["native_us"]}
 
@@ -757,6 +779,7 @@ def main():
             "draft_windowed_gbs_l2": win_gbs,
             "verify_gbs": ver_gbs,
             "device_status": status,
+            "read_stream_gbs_torch_sum": read_gbs,
         },
         "roofline": {"bound": "hbm", "achieved": ver_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": ver_gbs / hbm_peak, "traffic": verify_traffic(workload_desc(args)),
