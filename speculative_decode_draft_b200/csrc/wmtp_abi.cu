@@ -23,6 +23,8 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxRows = 64;
 constexpr int kMaxGammaMax = 16;
+constexpr int kMaxVerifyWaves = 8;      // CTAs per SM in turn for the tcgen05 verify of a batch
+constexpr int kMinTilesPerSplit = 16;   // extra waves only while full-capacity splits keep this many tiles
 constexpr size_t kWsAlign = 256;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -131,10 +133,18 @@ int ctas_per_sm_rt(int D, int NT) {
   return 1;
 }
 
-LaunchPlan make_plan(int sms, int B, int Hkv, long long rows_total, int D, int NT, long long max_tiles) {
+// `waves`: how many CTAs each SM runs in turn.  One wave splits the batch's
+// work evenly only when the sequences have similar lengths; with w = B waves
+// every sequence gets the same number of splits and each SM runs one CTA of
+// every sequence, so its total work follows the sum of the lengths whatever
+// they are (used by the tcgen05 verify, which is bound per SM by its MMA issue
+// chain; the bandwidth-bound kernels rebalance through the memory system).
+LaunchPlan make_plan(int sms, int B, int Hkv, long long rows_total, int D, int NT, long long max_tiles,
+                     int waves = 1) {
   LaunchPlan pl;
-  const long long slots = static_cast<long long>(sms) * ctas_per_sm_rt(D, NT);
+  const long long slots = static_cast<long long>(sms) * ctas_per_sm_rt(D, NT) * waves;
   long long per = slots / (static_cast<long long>(B) * Hkv);
+  if (waves > 1 && per > max_tiles / kMinTilesPerSplit) per = max_tiles / kMinTilesPerSplit;
   if (per < 1) per = 1;
   if (per > max_tiles) per = max_tiles;
   if (per < 1) per = 1;
@@ -255,7 +265,9 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
   const int rows = num_q * G;
   const int NT = (rows + 7) / 8;
   const long long rows_total = static_cast<long long>(B) * num_q * p->num_heads_q;
-  LaunchPlan pl = make_plan(info.sms, B, p->num_heads_kv, rows_total, D, NT, max_tiles < 1 ? 1 : max_tiles);
+  const bool tc = !RING && use_verify_tc(D, num_q, rows);
+  const int waves = tc ? (B < kMaxVerifyWaves ? B : kMaxVerifyWaves) : 1;
+  LaunchPlan pl = make_plan(info.sms, B, p->num_heads_kv, rows_total, D, NT, max_tiles < 1 ? 1 : max_tiles, waves);
   if (workspace == nullptr) {
     *workspace_bytes = pl.bytes;
     return WMTP_OK;
@@ -273,7 +285,7 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
   a.scale_log2 = scale_log2(p);
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_lse);
-  if (!RING && use_verify_tc(D, num_q, rows))
+  if (tc)
     s = launch_verify_tc(*tk, *tv, a, B, st);
   else
     s = launch_decode<RING>(D, NT, *tk, *tv, a, B, st);
