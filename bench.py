@@ -314,7 +314,9 @@ class Workload:
         self.workspace = torch.empty(max(
             w.workspace_bytes("full", self.p, self.B, max_pages=self.draft.max_pages),
             w.workspace_bytes("verify", self.p, self.B, num_q=self.gamma + 1, max_pages=self.layers[0].max_pages),
-            w.workspace_bytes("windowed", self.p, self.B)), dtype=torch.uint8, device=dev)
+            w.workspace_bytes("windowed", self.p, self.B),
+            w.workspace_bytes("windowed_paged", self.p, self.B, max_pages=self.draft.max_pages)),
+            dtype=torch.uint8, device=dev)
 
     # -- kernel launches of one step (for gpu_launches)
     def launches_per_step(self, arm: str) -> int:
@@ -717,6 +719,25 @@ def main():
     torch.cuda.synchronize()
     status = int(wk.status.item())
 
+    # the windowed draft read through the page table (no ring) over the draft
+    # layer's cache: ten calls captured in one CUDA graph, mean per call
+    win_paged_us = None
+    if not args.sweep:
+        wk.draft_cache.kv_len = wk.len_draft[args.warmup, 0]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(10):
+                w.draft_attn_windowed_paged(wk.p, wk.q_draft[args.warmup][0], wk.draft_cache, out=wk.o_draft,
+                                            lse=wk.l_draft, workspace=wk.workspace, status=wk.status)
+        g.replay()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record()
+        g.replay()
+        b1.record()
+        torch.cuda.synchronize()
+        win_paged_us = b0.elapsed_time(b1) * 1000.0 / 10
+        del g
+
     # a read-only streaming reference (torch's sum over 4 GiB; context for the
     # GB/s figures, not a peak the roofline divides by)
     read_gbs = None
@@ -732,6 +753,7 @@ def main():
             best = min(best, a0.elapsed_time(a1))
         read_gbs = big.numel() * 2 / (best * 1e-3) / 1e9
         del big
+    status = int(wk.status.item())  # including the extra windowed-paged calls
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -773,6 +795,7 @@ def main():
             "bytes_implied_ratio": (wk.gamma + wk.L) / wk.L,
             "draft_native_us": k_nat["draft"],
             "draft_windowed_us": k_win["draft"],
+            "draft_windowed_paged_us": win_paged_us,
             "verify_us_per_layer": k_win["verify"],
             "verify_us_per_layer_native_arm": k_nat["verify"],
             "draft_native_gbs": nat_gbs,

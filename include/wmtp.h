@@ -145,6 +145,26 @@ wmtp_status wmtp_draft_attn_full(const wmtp_params* params, int32_t batch, const
                                  int32_t* status_word, void* stream);
 
 /*
+ * wmtp_draft_attn_windowed_paged -- Windowed-MTP draft attention read through
+ * the page table, with no ring.
+ * Source: arxivlens view, Abstract (the draft attends a sink plus a sliding
+ * window); the same attended set as wmtp_draft_attn_windowed, for callers that
+ * keep the draft layer's full paged cache.  The window may change from call
+ * to call (params->window), which a fixed-capacity ring cannot follow.
+ *
+ * For every sequence b and query head h: o = softmax(sm_scale * K q) V over
+ * positions p < min(S, kv_len[b]) and max(S, kv_len[b] - W) <= p < kv_len[b]
+ * of the paged cache.  Only the pages holding those positions are read: at
+ * most ceil(S/64) + ceil(W/64) + 1 tiles of 64 tokens per sequence.
+ *   Arguments, layouts, workspace and errors as wmtp_draft_attn_full;
+ *   params->sinks >= 0 and params->window >= 1 (else WMTP_ERR_INVALID_ARG).
+ */
+wmtp_status wmtp_draft_attn_windowed_paged(const wmtp_params* params, int32_t batch, const void* q,
+                                           const wmtp_paged_kv* kv, void* out, int32_t out_fp32,
+                                           float* lse_out, void* workspace, size_t* workspace_bytes,
+                                           int32_t* status_word, void* stream);
+
+/*
  * wmtp_draft_attn_windowed -- Windowed-MTP draft attention over the ring.
  * Source: arxivlens view, Abstract (StreamingLLM-style sink plus window on the
  * draft only; the compact ring buffer); readpriors post "Your Million-Token

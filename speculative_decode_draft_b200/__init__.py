@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     PagedCache,
     Ring,
     draft_attn_full,
+    draft_attn_windowed_paged,
     draft_attn_windowed,
     new_status,
     paged_write,

@@ -32,6 +32,7 @@ EXPORTS = (
     "wmtp_version",
     "wmtp_draft_attn_full",
     "wmtp_draft_attn_windowed",
+    "wmtp_draft_attn_windowed_paged",
     "wmtp_ring_append",
     "wmtp_ring_reset",
     "wmtp_verify_attn",
@@ -114,6 +115,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.wmtp_draft_attn_full.restype = c_int32
     lib.wmtp_draft_attn_full.argtypes = [PP, c_int32, c_void_p, PK, c_void_p, c_int32, c_void_p,
                                          c_void_p, sz, i32p, c_void_p]
+    lib.wmtp_draft_attn_windowed_paged.restype = c_int32
+    lib.wmtp_draft_attn_windowed_paged.argtypes = [PP, c_int32, c_void_p, PK, c_void_p, c_int32, c_void_p,
+                                                   c_void_p, sz, i32p, c_void_p]
     lib.wmtp_verify_attn.restype = c_int32
     lib.wmtp_verify_attn.argtypes = [PP, c_int32, c_int32, c_void_p, PK, c_void_p, c_int32, c_void_p,
                                      c_void_p, sz, i32p, c_void_p]

@@ -159,6 +159,9 @@ def workspace_bytes(kind: str, p: L.Params, batch: int, num_q: int = 1, max_page
         if kind == "full":
             L.check(kind, lib.wmtp_draft_attn_full(byref(p), batch, None, byref(desc), None, 1, None, None,
                                                    byref(size), None, None))
+        elif kind == "windowed_paged":
+            L.check(kind, lib.wmtp_draft_attn_windowed_paged(byref(p), batch, None, byref(desc), None, 1, None,
+                                                             None, byref(size), None, None))
         else:
             L.check(kind, lib.wmtp_verify_attn(byref(p), batch, num_q, None, byref(desc), None, 1, None, None,
                                                byref(size), None, None))
@@ -178,6 +181,22 @@ def draft_attn_full(p: L.Params, q: torch.Tensor, cache: PagedCache, *, out_fp32
         return fn(byref(p), B, None if ws is None else q.data_ptr(), byref(desc), o, int(out_fp32), l, ws,
                   size, stat, st)
     return _run_attention("wmtp_draft_attn_full", call, (B, Hq, D), q.device, out_fp32, out, lse,
+                          workspace, status)
+
+
+def draft_attn_windowed_paged(p: L.Params, q: torch.Tensor, cache: PagedCache, *, out_fp32: bool = True,
+                              out=None, lse=None, workspace=None, status=None, stream=None):
+    """Windowed-MTP draft attention read through the page table (sink +
+    window positions of the paged cache, no ring): q ``[B, Hq, D]`` bf16."""
+    _need(q, BF16, "q")
+    B, Hq, D = q.shape
+    desc = cache.desc()
+    st = _stream(stream)
+
+    def call(fn, o, l, ws, _unused, size, stat):
+        return fn(byref(p), B, None if ws is None else q.data_ptr(), byref(desc), o, int(out_fp32), l, ws,
+                  size, stat, st)
+    return _run_attention("wmtp_draft_attn_windowed_paged", call, (B, Hq, D), q.device, out_fp32, out, lse,
                           workspace, status)
 
 

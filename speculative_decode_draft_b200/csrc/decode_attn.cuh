@@ -72,6 +72,9 @@ struct DecodeArgs {
   const int32_t* ring_tags;  // [B][R]
   const int32_t* ring_len;   // [B]
   int ring_slots, sinks, window;
+  // paged source only: 1 = attend the sink + window positions of the pages
+  // (the windowed draft read through the page table), 0 = every position
+  int paged_window;
   // outputs
   float* part_o;    // [B*num_q*Hq][nsplit][D]
   float* part_lse;  // [B*num_q*Hq][nsplit]
@@ -179,7 +182,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     n_tok = seq_len;
   }
-  const int ntiles = (n_tok + kTileTokens - 1) / kTileTokens;
+  // Windowed paged mode: the attended positions are [0, pw_sink_end) and
+  // [pw_lo_win, n_tok).  Tiles holding none of them are skipped: virtual tile v
+  // maps to tile v for the ns sink tiles, then to tw0 + (v - ns).
+  const bool pwin = !RING && a.paged_window != 0;
+  const int pw_sink_end = pwin ? min(a.sinks, n_tok) : n_tok;
+  const int pw_lo_win = pwin ? max(a.sinks, n_tok - a.window) : n_tok;
+  const int ns = pwin ? (pw_sink_end + kTileTokens - 1) / kTileTokens : 0;
+  const int tw0 = pwin ? max(ns, pw_lo_win / kTileTokens) : 0;
+  const int ntiles = pwin ? ns + max(0, (n_tok + kTileTokens - 1) / kTileTokens - tw0)
+                          : (n_tok + kTileTokens - 1) / kTileTokens;
+  auto tile_of = [&](int v) { return (!pwin || v < ns) ? v : tw0 + (v - ns); };
   const int tps = (ntiles + a.nsplit - 1) / a.nsplit;
   const int t_begin = min(split * tps, ntiles);
   const int t_end = min(t_begin + tps, ntiles);
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           set_status(a.status, kDevTimeout);
           break;
         }
-        const int tile = t_begin + k;
+        const int tile = tile_of(t_begin + k);
         const uint32_t kdst = sbase + Plan::kOffK + stage * Plan::kStageBytes;
         const uint32_t vdst = kdst + Plan::kTileBytes;
         const uint32_t fb = bar_full + 8 * stage;
@@ -330,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool got = ptx::mbar_wait(bar_full + 8 * stage, par);
     const uint32_t kst = sbase + Plan::kOffK + stage * Plan::kStageBytes;
     const uint32_t vst = kst + Plan::kTileBytes;
-    const int tile = t_begin + k;
+    const int tile = tile_of(t_begin + k);
     const int tok0 = tile * kTileTokens;
     const bool tile_ok = got && stage_flag[stage] != 0;
 
@@ -395,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- scale and mask; S^T element e: token g (+8 for e>=2), row 2*t4 + (e&1)
     const int tokA = tok0 + 16 * warp + g;
     const int tokB = tokA + 8;
-    bool need_mask = !tile_ok || RING || (tok0 + kTileTokens > first_masked_tok);
+    bool need_mask = !tile_ok || RING || pwin || (tok0 + kTileTokens > first_masked_tok);
     if (!need_mask) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -411,6 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tagB = (tokB < R) ? a.ring_tags[static_cast<size_t>(b) * R + tokB] : -1;
         okA = okA && tokA < n_tok && tagA >= 0 && tagA < seq_len && (tagA < sink_end || tagA >= lo_win);
         okB = okB && tokB < n_tok && tagB >= 0 && tagB < seq_len && (tagB < sink_end || tagB >= lo_win);
+      } else if (pwin) {
+        okA = okA && (tokA < pw_sink_end || (tokA >= pw_lo_win && tokA < n_tok));
+        okB = okB && (tokB < pw_sink_end || (tokB >= pw_lo_win && tokB < n_tok));
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)

@@ -383,7 +383,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool failed = false;
 
     for (int k = 0; k < my_tiles; ++k) {
-      const int stage = k % STAGES;
       const int sb = k & 1;
       // S(k) complete implies K(k) landed.  (The K ring itself is not waited
       // on here: its stage may already hold a later tile, so a parity wait on

@@ -294,11 +294,14 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
                         lse_out, st, true);
 }
 
+// `window`: attend only the sink + window positions of the pages (num_q 1).
 wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, const void* q,
                             const wmtp_paged_kv* kv, void* out, int32_t out_fp32, float* lse_out,
-                            void* workspace, size_t* workspace_bytes, int32_t* status_word, void* stream) {
+                            void* workspace, size_t* workspace_bytes, int32_t* status_word, void* stream,
+                            bool window = false) {
   wmtp_status s = check_params(p, num_q);
   if (s != WMTP_OK) return s;
+  if (window && (num_q != 1 || p->sinks < 0 || p->window < 1)) return WMTP_ERR_INVALID_ARG;
   if (batch < 0 || kv == nullptr || workspace_bytes == nullptr) return WMTP_ERR_INVALID_ARG;
   if (!supported_page(p->page_size)) return WMTP_ERR_UNSUPPORTED;
   if (kv->num_pages <= 0 || kv->max_pages <= 0) return WMTP_ERR_INVALID_ARG;
@@ -309,7 +312,12 @@ wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, 
     if (workspace == nullptr) *workspace_bytes = 0;
     return WMTP_OK;
   }
-  const long long max_tiles = (max_tokens + kTileTokens - 1) / kTileTokens;
+  long long max_tiles = (max_tokens + kTileTokens - 1) / kTileTokens;
+  if (window) {  // at most the sink tiles plus the tiles the window touches
+    const long long wt =
+        (p->sinks + kTileTokens - 1) / kTileTokens + (p->window + kTileTokens - 1) / kTileTokens + 1;
+    if (wt < max_tiles) max_tiles = wt;
+  }
   CUtensorMap tk, tv;
   bool ready = false;
   if (workspace != nullptr) {
@@ -332,6 +340,9 @@ wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, 
   a.num_pages = kv->num_pages;
   a.page_size = p->page_size;
   a.status = status_word;
+  a.paged_window = window ? 1 : 0;
+  a.sinks = p->sinks;
+  a.window = p->window;
   return run_attention<false>(p, batch, num_q, q, &tk, &tv, a, max_tiles, out, out_fp32, lse_out, workspace,
                               workspace_bytes, static_cast<cudaStream_t>(stream), ready);
 }
@@ -400,6 +411,14 @@ wmtp_status wmtp_draft_attn_full(const wmtp_params* params, int32_t batch, const
                                  void* stream) {
   return paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, workspace, workspace_bytes,
                          status_word, stream);
+}
+
+wmtp_status wmtp_draft_attn_windowed_paged(const wmtp_params* params, int32_t batch, const void* q,
+                                           const wmtp_paged_kv* kv, void* out, int32_t out_fp32,
+                                           float* lse_out, void* workspace, size_t* workspace_bytes,
+                                           int32_t* status_word, void* stream) {
+  return paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, workspace, workspace_bytes,
+                         status_word, stream, true);
 }
 
 wmtp_status wmtp_verify_attn(const wmtp_params* params, int32_t batch, int32_t num_q, const void* q,

@@ -336,6 +336,58 @@ def test_windowed_equals_full_when_window_covers_context():
     np.testing.assert_allclose(f64(ow), f64(of), atol=1e-5, rtol=0)
 
 
+# ---------------------------------------------------------------- windowed draft over pages
+@pytest.mark.parametrize("S,W,lens,P,D,G", [
+    (4, 256, [2049], 16, 64, 4),                 # tiny shapes
+    (4, 2048, [32769], 64, 256, 8),              # window inside a long history
+    (0, 100, [5000, 64], 64, 256, 8),            # no sinks; W not a multiple of 64
+    (200, 50, [100], 64, 256, 8),                # shorter than the sinks
+    (4, 2048, [1500, 2052], 64, 256, 8),         # window reaches the sinks: the full set
+    (64, 1000, [70000, 123, 64 * 37 + 5], 32, 256, 8),  # ragged batch, window start mid-page
+    (5, 130, [9000], 128, 256, 4),               # sinks and window share no tile boundary
+])
+def test_windowed_paged_vs_oracle(S, W, lens, P, D, G):
+    Hkv = 2
+    p = _params(G * Hkv, Hkv, D, P, S, W)
+    kv = _paged(91 + S, len(lens), Hkv, D, P, lens)
+    q = synth.queries(92 + W, (len(lens), G * Hkv, D), device=DEV)
+    status = w.new_status(DEV)
+    out, lse = w.draft_attn_windowed_paged(p, q, cache_of(kv), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kp, vp, pt, ln = _oracle_pools(kv)
+    scale = 1 / np.sqrt(D)
+    ref, ref_lse = oracle.draft_attn_windowed_paged(f64(q), kp, vp, pt, ln, P, S, W, scale)
+    assert_close(f64(out), ref, f"windowed paged S={S} W={W} lens={lens}")
+    assert_lse_close(f64(lse), ref_lse, f"windowed paged S={S} W={W}")
+    # the full set when the window reaches the sinks
+    if all(n <= S + W for n in lens):
+        of, _ = w.draft_attn_full(p, q, cache_of(kv))
+        np.testing.assert_allclose(f64(out), f64(of), atol=1e-5, rtol=0)
+
+
+def test_windowed_paged_window_changes_per_call():
+    # an adaptive window: the same cache read with a different W on each call
+    S, D, G, Hkv, P = 4, 256, 8, 2, 64
+    lens = [40000]
+    kv = _paged(95, 1, Hkv, D, P, lens)
+    q = synth.queries(96, (1, G * Hkv, D), device=DEV)
+    kp, vp, pt, ln = _oracle_pools(kv)
+    for W in (64, 1000, 4096, 40000):
+        p = _params(G * Hkv, Hkv, D, P, S, W)
+        out, _ = w.draft_attn_windowed_paged(p, q, cache_of(kv))
+        ref, _ = oracle.draft_attn_windowed_paged(f64(q), kp, vp, pt, ln, P, S, W, 1 / 16)
+        assert_close(f64(out), ref, f"windowed paged W={W}")
+
+
+def test_windowed_paged_rejects_bad_window():
+    p = _params(16, 2, 256, 64, 4, 0)
+    kv = _paged(97, 1, 2, 256, 64, [100])
+    q = synth.queries(98, (1, 16, 256), device=DEV)
+    with pytest.raises(L.WmtpError):
+        w.draft_attn_windowed_paged(p, q, cache_of(kv))
+
+
 # ---------------------------------------------------------------- device status
 def test_bad_page_table_and_length_set_status():
     p = _params(8, 1, 64, 16)
