@@ -471,10 +471,10 @@ def cores_used():
 # hashes to the value it was captured on, and only for that workload.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "ae451fa4389a6245c14ea9f272014f41705bd3f9e1cf4cd165a8fdd9010609f1",
+    "sha256": "7f8dd707a0c30faf02c29a42c549ca312f84b295b00b01df44a1ce621af19e2e",
     "workload": "1m: batch 1, 16q/2kv heads, D=256, page 64, ctx 1048576, S=4, W=4096, gamma=3, 10 verify layers",
-    # mean of two captured launches: 2,147,830,528 + 3,226,880 and 2,147,822,848 + 264,960 bytes
-    "bytes": 2149572608,
+    # mean of two captured launches: 2,148,118,784 + 3,054,592 and 2,147,827,712 + 401,664 bytes
+    "bytes": 2149701376,
 }
 
 
@@ -652,6 +652,7 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     if args.sweep:
         return run_sweep(args, rank, world, dev)
+    free_bytes, _ = torch.cuda.mem_get_info()  # before the workload's own buffers
     wk = Workload(args, rank, dev)
     stream = torch.cuda.current_stream()
 
@@ -755,6 +756,15 @@ def main():
         del big
     status = int(wk.status.item())  # including the extra windowed-paged calls
 
+    # the capacity side: requests of this context that the device's free
+    # memory holds as KV, with the draft layer paged (native) or as a ring
+    adm = {arm: w.plan_admission(wk.p, wk.n0, wk.L, 1, arm == "windowed", free_bytes)
+           for arm in ("native", "windowed")}
+    admission = {"kv_budget_bytes": free_bytes, "context": wk.n0, "target_layers": wk.L, "draft_layers": 1,
+                 "native_requests": adm["native"]["max_requests"],
+                 "windowed_requests": adm["windowed"]["max_requests"],
+                 "reclaimed_fraction": 1 - adm["windowed"]["bytes_per_request"] / adm["native"]["bytes_per_request"]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_step_model(args, 524288, repeats=2)
@@ -803,6 +813,7 @@ def main():
             "verify_gbs": ver_gbs,
             "device_status": status,
             "read_stream_gbs_torch_sum": read_gbs,
+            "admission": admission,
         },
         "roofline": {"bound": "hbm", "achieved": ver_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": ver_gbs / hbm_peak, "traffic": verify_traffic(workload_desc(args)),

@@ -9,6 +9,7 @@ package is the thin PyTorch binding of that library.
 from ._lib import EXPORTS, WmtpError, load  # noqa: F401
 from .api import (  # noqa: F401
     PagedCache,
+    PagePool,
     Ring,
     draft_attn_full,
     draft_attn_windowed_paged,
@@ -16,6 +17,7 @@ from .api import (  # noqa: F401
     new_status,
     paged_write,
     params,
+    plan_admission,
     ring_append,
     ring_reset,
     splitkv_combine,

@@ -39,6 +39,12 @@ EXPORTS = (
     "wmtp_splitkv_combine",
     "wmtp_paged_write",
     "wmtp_draft_attn_full_noalloc",
+    "wmtp_pool_create",
+    "wmtp_pool_destroy",
+    "wmtp_pool_free_count",
+    "wmtp_pool_alloc",
+    "wmtp_pool_release",
+    "wmtp_plan_admission",
 )
 
 # Size of the fixed scratch array behind wmtp_draft_attn_full_noalloc.
@@ -80,6 +86,17 @@ class RingDesc(ctypes.Structure):
         ("undo_v", c_void_p),
         ("undo_tags", c_void_p),
         ("batch", c_int32),
+    ]
+
+
+class Admission(ctypes.Structure):
+    _fields_ = [
+        ("pages_per_layer", ctypes.c_int64),
+        ("page_bytes", ctypes.c_int64),
+        ("target_bytes", ctypes.c_int64),
+        ("draft_bytes", ctypes.c_int64),
+        ("bytes_per_request", ctypes.c_int64),
+        ("max_requests", ctypes.c_int64),
     ]
 
 
@@ -138,6 +155,19 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.wmtp_draft_attn_full_noalloc.restype = c_int32
     lib.wmtp_draft_attn_full_noalloc.argtypes = [PP, c_int32, c_void_p, PK, c_void_p, c_int32, c_void_p,
                                                  i32p, c_void_p]
+    lib.wmtp_pool_create.restype = c_int32
+    lib.wmtp_pool_create.argtypes = [c_int32, POINTER(c_void_p)]
+    lib.wmtp_pool_destroy.restype = None
+    lib.wmtp_pool_destroy.argtypes = [c_void_p]
+    lib.wmtp_pool_free_count.restype = c_int32
+    lib.wmtp_pool_free_count.argtypes = [c_void_p]
+    lib.wmtp_pool_alloc.restype = c_int32
+    lib.wmtp_pool_alloc.argtypes = [c_void_p, c_int32, c_void_p]
+    lib.wmtp_pool_release.restype = c_int32
+    lib.wmtp_pool_release.argtypes = [c_void_p, c_int32, c_void_p]
+    lib.wmtp_plan_admission.restype = c_int32
+    lib.wmtp_plan_admission.argtypes = [PP, ctypes.c_int64, c_int32, c_int32, c_int32, ctypes.c_int64,
+                                        POINTER(Admission)]
     if path is None:
         _lib = lib
     return lib

@@ -287,3 +287,48 @@ def paged_write(p: L.Params, cache: PagedCache, pos0: torch.Tensor, k_new: torch
 def new_status(device) -> torch.Tensor:
     """A zeroed device status word for the ``status=`` arguments."""
     return torch.zeros(1, dtype=I32, device=device)
+
+
+# ---------------------------------------------------------------- serving-side helpers (host only)
+class PagePool:
+    """Free-list allocator over the page indices of one pool tensor
+    (``wmtp_pool_*``; host memory only)."""
+
+    def __init__(self, num_pages: int):
+        self._lib = L.load()
+        h = c_void_p()
+        L.check("wmtp_pool_create", self._lib.wmtp_pool_create(int(num_pages), byref(h)))
+        self._h = h
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.wmtp_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    @property
+    def free_count(self) -> int:
+        return int(self._lib.wmtp_pool_free_count(self._h))
+
+    def alloc(self, n: int) -> list[int]:
+        """``n`` page indices; raises WmtpError (WMTP_ERR_WORKSPACE) if fewer are free."""
+        buf = (ctypes.c_int32 * max(int(n), 1))()
+        L.check("wmtp_pool_alloc", self._lib.wmtp_pool_alloc(self._h, int(n), buf))
+        return list(buf[:int(n)])
+
+    def release(self, pages) -> None:
+        pages = list(pages)
+        buf = (ctypes.c_int32 * max(len(pages), 1))(*pages)
+        L.check("wmtp_pool_release", self._lib.wmtp_pool_release(self._h, len(pages), buf))
+
+
+def plan_admission(p: L.Params, context: int, target_layers: int, draft_layers: int, windowed: bool,
+                   kv_budget_bytes: int) -> dict:
+    """Per-request KV footprint and the requests a budget admits (``wmtp_plan_admission``)."""
+    out = L.Admission()
+    L.check("wmtp_plan_admission", L.load().wmtp_plan_admission(
+        byref(p), int(context), int(target_layers), int(draft_layers), int(bool(windowed)),
+        int(kv_budget_bytes), byref(out)))
+    return {name: int(getattr(out, name)) for name, _ in L.Admission._fields_}
