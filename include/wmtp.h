@@ -18,7 +18,12 @@
  *   host during the call and may be freed when it returns.  The library never
  *   allocates device memory.
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- *   default stream) and never synchronise the host.
+ *   default stream) and never synchronise the host.  The attention kernels
+ *   are launched as programmatic dependents of the work before them on the
+ *   stream: their set-up may overlap its tail, but they read no global memory
+ *   before it has completed, so stream order holds for every input.  The calls
+ *   can be captured in CUDA graphs (the first call on a device must come
+ *   before any capture: it sets kernel attributes).
  * - Host-detectable argument errors return a negative wmtp_status before
  *   anything is launched.
  * - Device-detected problems (a page-table entry outside the pool, a length
