@@ -238,6 +238,30 @@ wmtp_status wmtp_verify_attn(const wmtp_params* params, int32_t batch, int32_t n
                              size_t* workspace_bytes, int32_t* status_word, void* stream);
 
 /*
+ * wmtp_verify_attn_slice -- verify attention over one slice of each
+ * sequence's context (context parallelism).
+ * Not on the pages as such: the pages verify on one GPU.  A sequence whose
+ * context is spread over several caches (one per GPU, each holding a
+ * contiguous range of positions) is verified by calling this on every slice
+ * and merging the (out, lse) pairs with wmtp_splitkv_combine, which is exact
+ * because softmax attention over a union of disjoint key sets is the
+ * log-sum-exp merge of the attentions over each set.
+ *
+ * As wmtp_verify_attn, except that query i of sequence b attends the
+ * positions p < kv_len[b] of this cache with p <= q_pos0[b] + i, where
+ * q_pos0[b] (device int32, required) is the position of query 0 counted from
+ * the slice's first token: for a slice starting at global position s of a
+ * sequence whose num_q queries sit at n - num_q .. n - 1, q_pos0 = n - num_q - s.
+ * A slice entirely before the queries (q_pos0 >= kv_len) is attended in
+ * full; a query that sees no position of the slice gets out = 0, lse = -inf.
+ * kv_len[b] may be smaller than num_q.
+ */
+wmtp_status wmtp_verify_attn_slice(const wmtp_params* params, int32_t batch, int32_t num_q, const void* q,
+                                   const wmtp_paged_kv* kv, const int32_t* q_pos0, void* out, int32_t out_fp32,
+                                   float* lse_out, void* workspace, size_t* workspace_bytes, int32_t* status_word,
+                                   void* stream);
+
+/*
  * wmtp_splitkv_combine -- merge split-KV partial attention results.
  * Not on the pages: the standard log-sum-exp identity behind split-KV
  * (flash-decoding) decode attention, needed to spread one sequence over the

@@ -201,12 +201,25 @@ def draft_attn_windowed_paged(p: L.Params, q: torch.Tensor, cache: PagedCache, *
 
 
 def verify_attn(p: L.Params, q: torch.Tensor, cache: PagedCache, *, out_fp32: bool = True, out=None,
-                lse=None, workspace=None, status=None, stream=None):
-    """Verify attention: q ``[B, num_q, Hq, D]`` bf16 -> (out, lse)."""
+                lse=None, workspace=None, status=None, stream=None, q_pos0: torch.Tensor | None = None):
+    """Verify attention: q ``[B, num_q, Hq, D]`` bf16 -> (out, lse).
+
+    ``q_pos0`` (int32 ``[B]``): the cache holds a slice of each sequence and
+    query 0 sits at this position counted from the slice's first token
+    (``wmtp_verify_attn_slice``); None means the cache holds the whole context
+    and the queries are its last ``num_q`` positions."""
     _need(q, BF16, "q")
     B, Qn, Hq, D = q.shape
     desc = cache.desc()
     st = _stream(stream)
+    if q_pos0 is not None:
+        _need(q_pos0, I32, "q_pos0", q.device)
+
+        def call_slice(fn, o, l, ws, _unused, size, stat):
+            return fn(byref(p), B, Qn, None if ws is None else q.data_ptr(), byref(desc),
+                      None if ws is None else q_pos0.data_ptr(), o, int(out_fp32), l, ws, size, stat, st)
+        return _run_attention("wmtp_verify_attn_slice", call_slice, (B, Qn, Hq, D), q.device, out_fp32, out,
+                              lse, workspace, status)
 
     def call(fn, o, l, ws, _unused, size, stat):
         return fn(byref(p), B, Qn, None if ws is None else q.data_ptr(), byref(desc), o, int(out_fp32), l,

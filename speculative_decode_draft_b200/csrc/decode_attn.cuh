@@ -75,6 +75,9 @@ struct DecodeArgs {
   // paged source only: 1 = attend the sink + window positions of the pages
   // (the windowed draft read through the page table), 0 = every position
   int paged_window;
+  // paged source only: [B] position of query 0 counted from this cache's first
+  // token (a slice of a longer sequence), or NULL for kv_len - num_q
+  const int32_t* q_pos0;
   // outputs
   float* part_o;    // [B*num_q*Hq][nsplit][D]
   float* part_lse;  // [B*num_q*Hq][nsplit]
@@ -176,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     n_tok = min(seq_len, a.ring_slots);
   } else {
     seq_len = a.kv_len[b];
-    if (seq_len != 0 && (seq_len < a.num_q || seq_len > a.max_pages * a.page_size)) {
+    if (seq_len != 0 &&
+        ((a.q_pos0 == nullptr && seq_len < a.num_q) || seq_len < 0 || seq_len > a.max_pages * a.page_size)) {
       if (threadIdx.x == 0 && split == 0 && kvh == 0) set_status(a.status, kDevLenOob);
       seq_len = 0;
     }
@@ -193,6 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = pwin ? ns + max(0, (n_tok + kTileTokens - 1) / kTileTokens - tw0)
                           : (n_tok + kTileTokens - 1) / kTileTokens;
   auto tile_of = [&](int v) { return (!pwin || v < ns) ? v : tw0 + (v - ns); };
+  // position of query 0 in this cache: query i attends positions <= q_first + i
+  const int q_first = (!RING && a.q_pos0 != nullptr) ? a.q_pos0[b] : n_tok - a.num_q;
   const int tps = (ntiles + a.nsplit - 1) / a.nsplit;
   const int t_begin = min(split * tps, ntiles);
   const int t_end = min(t_begin + tps, ntiles);
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (RING || row >= a.rows)
         lim[nt][j] = n_tok;
       else
-        lim[nt][j] = n_tok - a.num_q + row / a.G + 1;
+        lim[nt][j] = min(n_tok, q_first + row / a.G + 1);
     }
 
   float o_acc[kMT][NT][4];
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   const int dbase = warp * (D / 4);
-  const int first_masked_tok = RING ? -1 : (n_tok - a.num_q + 1);  // tokens >= this may be masked
+  const int first_masked_tok = RING ? -1 : min(n_tok, q_first + 1);  // tokens >= this may be masked
 
   for (int k = 0; k < my_tiles; ++k) {
     const int stage = k % STAGES;

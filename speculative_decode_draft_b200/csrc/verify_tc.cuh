@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ---- token range of this split
   int n_tok = a.kv_len[b];
-  if (n_tok != 0 && (n_tok < a.num_q || n_tok > a.max_pages * a.page_size)) {
+  if (n_tok != 0 &&
+      ((a.q_pos0 == nullptr && n_tok < a.num_q) || n_tok < 0 || n_tok > a.max_pages * a.page_size)) {
     if (threadIdx.x == 0 && split == 0 && kvh == 0) set_status(a.status, kDevLenOob);
     n_tok = 0;
   }
@@ -376,8 +377,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_q_ready);
     }
-    const int lim = row_active ? n_tok - a.num_q + row / a.G + 1 : n_tok;  // causal limit of this row
-    const int first_masked_tok = n_tok - a.num_q + 1;
+    // query i attends positions <= q_first + i of this cache (q_first is
+    // kv_len - num_q unless the call covers a slice of a longer sequence)
+    const int q_first = a.q_pos0 != nullptr ? a.q_pos0[b] : n_tok - a.num_q;
+    const int lim = row_active ? min(n_tok, q_first + row / a.G + 1) : n_tok;  // causal limit of this row
+    const int first_masked_tok = min(n_tok, q_first + 1);
     float m_ref = -INFINITY;  // reference maximum (log2 units)
     float l_run = 0.f;
     bool failed = false;

@@ -298,7 +298,7 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
 wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, const void* q,
                             const wmtp_paged_kv* kv, void* out, int32_t out_fp32, float* lse_out,
                             void* workspace, size_t* workspace_bytes, int32_t* status_word, void* stream,
-                            bool window = false) {
+                            bool window = false, const int32_t* q_pos0 = nullptr) {
   wmtp_status s = check_params(p, num_q);
   if (s != WMTP_OK) return s;
   if (window && (num_q != 1 || p->sinks < 0 || p->window < 1)) return WMTP_ERR_INVALID_ARG;
@@ -341,6 +341,7 @@ wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, 
   a.page_size = p->page_size;
   a.status = status_word;
   a.paged_window = window ? 1 : 0;
+  a.q_pos0 = q_pos0;
   a.sinks = p->sinks;
   a.window = p->window;
   return run_attention<false>(p, batch, num_q, q, &tk, &tv, a, max_tiles, out, out_fp32, lse_out, workspace,
@@ -419,6 +420,15 @@ wmtp_status wmtp_draft_attn_windowed_paged(const wmtp_params* params, int32_t ba
                                            int32_t* status_word, void* stream) {
   return paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, workspace, workspace_bytes,
                          status_word, stream, true);
+}
+
+wmtp_status wmtp_verify_attn_slice(const wmtp_params* params, int32_t batch, int32_t num_q, const void* q,
+                                   const wmtp_paged_kv* kv, const int32_t* q_pos0, void* out, int32_t out_fp32,
+                                   float* lse_out, void* workspace, size_t* workspace_bytes, int32_t* status_word,
+                                   void* stream) {
+  if (workspace != nullptr && q_pos0 == nullptr) return WMTP_ERR_INVALID_ARG;
+  return paged_attention(params, batch, num_q, q, kv, out, out_fp32, lse_out, workspace, workspace_bytes,
+                         status_word, stream, false, q_pos0);
 }
 
 wmtp_status wmtp_verify_attn(const wmtp_params* params, int32_t batch, int32_t num_q, const void* q,
