@@ -19,7 +19,7 @@
 // each softmax warp owns a quarter of them.
 //
 // Roles: warp 0 streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
-// into two STAGES-deep shared-memory rings with TMA, one lane per ring: a K
+// into two shared-memory rings (KS and VS tiles deep) with TMA, one lane per ring: a K
 // tile is released as soon as its S = Q K^T has completed, a V tile only
 // after its O += P V, so K loads run ahead of the softmax instead of waiting
 // for the slower PV of the same tile; warp 1 allocates the tensor
@@ -63,22 +63,26 @@ constexpr uint32_t kColS = 128;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;   // lazy rescale threshold (log2 units)
 
-template <int STAGES>
+template <int KS, int VS>
 struct TcPlan {
   static constexpr int kChunkBytes = 64 * 128;           // 64 tokens x 128 B
   static constexpr int kTileBytes = 4 * kChunkBytes;      // one K or V tile, D = 256
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kOffK = 0;
-  static constexpr int kOffBar = STAGES * kStageBytes;
-  // k_full[S], k_empty[S], v_full[S], v_empty[S], v_ready[S], s_full[2],
-  // p_full[2], o_done, mma_final
-  static constexpr int kNumBars = 5 * STAGES + 7;
+  static constexpr int kOffK = 0;                         // K ring: KS tiles
+  static constexpr int kOffV = KS * kTileBytes;           // V ring: VS tiles
+  static constexpr int kOffBar = (KS + VS) * kTileBytes;
+  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], v_ready[VS], s_full[2],
+  // p_full[2], o_done, mma_final, q_ready
+  static constexpr int kNumBars = 2 * KS + 3 * VS + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort
   static constexpr int kBytes = kOffMisc + 8;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-constexpr int kTcStages = 3;
+// Depths of the K and V rings (64-token tiles).  K tiles leave as soon as QK
+// has read them and V tiles only after the softmax and PV, yet 2 + 4 measured
+// slower than 3 + 3 on B200 (398-404 against 393-396 us per 1M layer).
+constexpr int kTcKStages = 3;
+constexpr int kTcVStages = 3;
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -91,11 +95,11 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
   }
 }
 
-template <int STAGES>
+template <int KS, int VS>
 __global__ void __launch_bounds__(kTcThreads, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const DecodeArgs a) {
-  using Plan = TcPlan<STAGES>;
+  using Plan = TcPlan<KS, VS>;
   constexpr int D = 256;
 
   extern __shared__ uint8_t smem_raw[];
@@ -104,11 +108,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t sbase = ptx::smem_addr(smem);
   const uint32_t bar0 = sbase + Plan::kOffBar;
   const uint32_t bar_k_full = bar0;
-  const uint32_t bar_k_empty = bar0 + 8 * STAGES;
-  const uint32_t bar_v_full = bar0 + 16 * STAGES;
-  const uint32_t bar_v_empty = bar0 + 24 * STAGES;
-  const uint32_t bar_v_ready = bar0 + 32 * STAGES;
-  const uint32_t bar_s_full = bar0 + 40 * STAGES;
+  const uint32_t bar_k_empty = bar_k_full + 8 * KS;
+  const uint32_t bar_v_full = bar_k_empty + 8 * KS;
+  const uint32_t bar_v_empty = bar_v_full + 8 * VS;
+  const uint32_t bar_v_ready = bar_v_empty + 8 * VS;
+  const uint32_t bar_s_full = bar_v_ready + 8 * VS;
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_o_done = bar_p_full + 16;
   const uint32_t bar_final = bar_o_done + 8;
@@ -124,9 +128,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ---- set-up: barriers and tensor memory
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < KS; ++s) {
       ptx::mbar_init(bar_k_full + 8 * s, 1);
       ptx::mbar_init(bar_k_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       ptx::mbar_init(bar_v_full + 8 * s, 1);
       ptx::mbar_init(bar_v_empty + 8 * s, 1);
       ptx::mbar_init(bar_v_ready + 8 * s, 4);
@@ -163,7 +169,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int my_tiles = t_end - t_begin;
   // start the page-table reads of the first tiles now; the producers' own
   // loads then hit L2
-  if (warp == 0 && lane < STAGES && lane < my_tiles) {
+  if (warp == 0 && lane < VS && lane < my_tiles) {
     const int* pte = a.page_table + static_cast<size_t>(b) * a.max_pages +
                      ((t_begin + lane) * kTileTokens) / a.page_size;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(pte));
@@ -195,17 +201,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int oob_z = a.num_pages * a.Hkv;  // past the tensor: zero fill
       const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
       const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
-      const uint32_t ring = sbase + Plan::kOffK + (is_k ? 0 : Plan::kTileBytes);
+      const uint32_t ring = sbase + (is_k ? Plan::kOffK : Plan::kOffV);
+      const int nst = is_k ? KS : VS;  // stages of this lane's ring
       int issued = 0;
       for (int k = 0; k < my_tiles; ++k) {
-        const int stage = k % STAGES;
-        if (!tc_wait(bar_empty + 8 * stage, ((k / STAGES) & 1) ^ 1, abort_flag)) {
+        const int stage = k % nst;
+        if (!tc_wait(bar_empty + 8 * stage, ((k / nst) & 1) ^ 1, abort_flag)) {
           if (*abort_flag == 0) set_status(a.status, kDevTimeout);
           *abort_flag = 1;
           break;
         }
         const int tok0 = (t_begin + k) * kTileTokens;
-        const uint32_t dst = ring + stage * Plan::kStageBytes;
+        const uint32_t dst = ring + stage * Plan::kTileBytes;
         const uint32_t fb = bar_full + 8 * stage;
         int zs[4], ys[4];
         int valid = 1;
@@ -235,8 +242,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // no copy may still be writing shared memory when the CTA exits (after
       // an abort the consumers stop early): wait, bounded, for the last load
       // of each stage
-      for (int k = max(issued - STAGES, 0); k < issued; ++k)
-        if (!ptx::mbar_wait(bar_full + 8 * (k % STAGES), (k / STAGES) & 1)) set_status(a.status, kDevTimeout);
+      for (int k = max(issued - nst, 0); k < issued; ++k)
+        if (!ptx::mbar_wait(bar_full + 8 * (k % nst), (k / nst) & 1)) set_status(a.status, kDevTimeout);
     }
     return;
   }
@@ -246,16 +253,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int cw = warp - 6;  // one 8 KB column chunk (64 head dims) of the V tile per warp
     uint32_t vexp = 0;        // per-half maximum of the bf16 exponent fields seen
     for (int k = 0; k < my_tiles; ++k) {
-      const int stage = k % STAGES;
-      if (!__all_sync(0xffffffffu, tc_wait(bar_v_full + 8 * stage, (k / STAGES) & 1, abort_flag))) {
+      const int stage = k % VS;
+      if (!__all_sync(0xffffffffu, tc_wait(bar_v_full + 8 * stage, (k / VS) & 1, abort_flag))) {
         if (lane == 0) set_status(a.status, kDevTimeout);
         *abort_flag = 1;
         break;
       }
       const int tok0 = (t_begin + k) * kTileTokens;
       const int rows_valid = min(kTileTokens, n_tok - tok0);
-      const uint32_t chunk = sbase + Plan::kOffK + stage * Plan::kStageBytes + Plan::kTileBytes +
-                             cw * Plan::kChunkBytes;
+      const uint32_t chunk = sbase + Plan::kOffV + stage * Plan::kTileBytes + cw * Plan::kChunkBytes;
 #pragma unroll 4
       for (int u = lane; u < Plan::kChunkBytes / 16; u += 32) {
         const uint32_t addr = chunk + 16 * u;
@@ -296,9 +302,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // descriptor start addresses are in 16-byte units in the low bits, so
       // moving an operand by n bytes adds n >> 4 to the descriptor
       const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
-      const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK + Plan::kTileBytes, Plan::kChunkBytes, 1024);
+      const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffV, Plan::kChunkBytes, 1024);
       auto issue_qk = [&](int k) {
-        const uint64_t kd = k_desc0 + (static_cast<uint64_t>((k % STAGES) * Plan::kStageBytes) >> 4);
+        const uint64_t kd = k_desc0 + (static_cast<uint64_t>((k % KS) * Plan::kTileBytes) >> 4);
         const uint32_t d_tmem = tmem_base + kColS + (k & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -306,7 +312,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
         }
         tc::commit(bar_s_full + 8 * (k & 1));
-        tc::commit(bar_k_empty + 8 * (k % STAGES));
+        tc::commit(bar_k_empty + 8 * (k % KS));
       };
       // Q is staged into TMEM by the softmax warps while the first K/V tiles
       // are in flight
@@ -319,23 +325,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (k + 1 < my_tiles) {
           // the S/P buffer of tile k+1 last held P(k-1), read by PV(k-1),
           // which was issued earlier and runs first
-          ok = tc_wait(bar_k_full + 8 * ((k + 1) % STAGES), ((k + 1) / STAGES) & 1, abort_flag);
+          ok = tc_wait(bar_k_full + 8 * ((k + 1) % KS), ((k + 1) / KS) & 1, abort_flag);
           if (!ok) break;
           tc::fence_after_sync();
           issue_qk(k + 1);
         }
         ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag) &&
-             tc_wait(bar_v_ready + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag);
+             tc_wait(bar_v_ready + 8 * (k % VS), (k / VS) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
-        const uint64_t vd = v_desc0 + (static_cast<uint64_t>((k % STAGES) * Plan::kStageBytes) >> 4);
+        const uint64_t vd = v_desc0 + (static_cast<uint64_t>((k % VS) * Plan::kTileBytes) >> 4);
         const uint32_t p_tmem = tmem_base + kColS + (k & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
           const uint64_t bd = vd + (static_cast<uint32_t>(kk * 2048) >> 4);
           tc::mma_ts(tmem_base + kColO, p_tmem + 8 * kk, bd, kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::commit(bar_v_empty + 8 * (k % STAGES));
+        tc::commit(bar_v_empty + 8 * (k % VS));
         tc::commit(bar_o_done);
       }
       if (!ok) {

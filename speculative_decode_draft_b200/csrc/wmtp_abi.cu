@@ -211,9 +211,9 @@ wmtp_status launch_decode(int D, int NT, const CUtensorMap& tk, const CUtensorMa
 
 wmtp_status launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
                              cudaStream_t st) {
-  constexpr int alloc = TcPlan<kTcStages>::kAlloc;
+  constexpr int alloc = TcPlan<kTcKStages, kTcVStages>::kAlloc;
   static_assert(alloc <= kSmemLimit, "shared-memory plan exceeds the sm_100 per-block limit");
-  auto kern = verify_tc_kernel<kTcStages>;
+  auto kern = verify_tc_kernel<kTcKStages, kTcVStages>;
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
