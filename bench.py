@@ -471,10 +471,10 @@ def cores_used():
 # hashes to the value it was captured on, and only for that workload.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "7f8dd707a0c30faf02c29a42c549ca312f84b295b00b01df44a1ce621af19e2e",
+    "sha256": "de533333a847358c9f82325a5a119c0ee4141083d75920283861a55c13863767",
     "workload": "1m: batch 1, 16q/2kv heads, D=256, page 64, ctx 1048576, S=4, W=4096, gamma=3, 10 verify layers",
-    # mean of two captured launches: 2,148,118,784 + 3,054,592 and 2,147,827,712 + 401,664 bytes
-    "bytes": 2149701376,
+    # mean of two captured launches: 2,147,901,440 + 5,658,368 and 2,147,835,136 + 195,328 bytes
+    "bytes": 2150795136,
 }
 
 
