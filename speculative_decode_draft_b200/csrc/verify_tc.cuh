@@ -23,9 +23,10 @@
 // tile is released as soon as its S = Q K^T has completed, a V tile only
 // after its O += P V, so K loads run ahead of the softmax instead of waiting
 // for the slower PV of the same tile; warp 1 allocates the tensor
-// memory and one lane issues every MMA (S = Q K^T as M=64, N=64 with K from
-// shared memory, K-major; O += P V as M=64, N=256 with V read MN-major
-// straight from the TMA tile); warps 2..5 run the softmax, one thread per
+// memory and one lane issues S = Q K^T (M=64, N=64, K from shared memory,
+// K-major) while one lane of warp 10 issues O += P V (M=64, N=256, V read
+// MN-major straight from the TMA tile): a lane issues a small tcgen05.mma
+// only every ~66 cycles, so two issuing lanes keep the tensor pipe busier; warps 2..5 run the softmax, one thread per
 // row: the row's scores come out of TMEM, the maximum and sum are taken
 // inside the thread, and P goes back into TMEM in fp16; warps 6..9 convert
 // each landed V tile in place from bf16 to fp16 (and zero its rows past the
@@ -55,7 +56,8 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 320;       // producers, MMA, 4 softmax warps, 4 V converter warps
+constexpr int kTcThreads = 352;       // producers, QK issuer, 4 softmax warps, 4 V converter warps, PV issuer
+constexpr int kPvWarp = 10;
 constexpr int kBarTmem = 3;           // named barrier: MMA + softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;
@@ -71,8 +73,8 @@ struct TcPlan {
   static constexpr int kOffV = KS * kTileBytes;           // V ring: VS tiles
   static constexpr int kOffBar = (KS + VS) * kTileBytes;
   // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], v_ready[VS], s_full[2],
-  // p_full[2], o_done, mma_final, q_ready
-  static constexpr int kNumBars = 2 * KS + 3 * VS + 7;
+  // p_full[2], o_done, mma_final, q_ready, pv_done[2]
+  static constexpr int kNumBars = 2 * KS + 3 * VS + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort
   static constexpr int kBytes = kOffMisc + 8;
   static constexpr int kAlloc = kBytes + 1024;
@@ -117,6 +119,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_o_done = bar_p_full + 16;
   const uint32_t bar_final = bar_o_done + 8;
   const uint32_t bar_q_ready = bar_final + 8;
+  const uint32_t bar_pv_done = bar_q_ready + 8;  // [2]: PV of the tiles using S/P buffer 0 / 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
 
@@ -142,7 +145,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::mbar_init(bar_p_full + 8 * i, 4);
     }
     ptx::mbar_init(bar_o_done, 1);
-    ptx::mbar_init(bar_final, 1);
+    ptx::mbar_init(bar_final, 2);  // one commit from each MMA-issuing lane
+    ptx::mbar_init(bar_pv_done, 1);
+    ptx::mbar_init(bar_pv_done + 8, 1);
     ptx::mbar_init(bar_q_ready, 4);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // =================================================================== V converters
-  if (warp >= 6) {
+  if (warp >= 6 && warp < kPvWarp) {
     const int cw = warp - 6;  // one 8 KB column chunk (64 head dims) of the V tile per warp
     uint32_t vexp = 0;        // per-half maximum of the bf16 exponent fields seen
     for (int k = 0; k < my_tiles; ++k) {
@@ -292,44 +297,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return;
   }
 
-  // =================================================================== MMA issuer
-  if (warp == 1) {
+  // =================================================================== PV issuer
+  // O += P(k) V(k) for every tile, issued by its own lane: a single lane
+  // issues a small tcgen05.mma only every ~66 cycles, so the QK and PV
+  // streams run from two lanes and overlap in the tensor pipe.
+  if (warp == kPvWarp) {
     if (lane == 0 && my_tiles > 0) {
-      // M = 64: the rows never exceed 64, and an M=64 MMA costs the same
-      // issue time as M=128 for half the tensor work (and power)
-      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(64, 64, 0, 0);    // A (Q, TMEM), B (K) K-major
       constexpr uint32_t kIdescPV = tc::idesc_f16_f32(64, 256, 0, 1);    // A (P, TMEM), B (V) MN-major, fp16
-      // descriptor start addresses are in 16-byte units in the low bits, so
-      // moving an operand by n bytes adds n >> 4 to the descriptor
-      const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
       const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffV, Plan::kChunkBytes, 1024);
-      auto issue_qk = [&](int k) {
-        const uint64_t kd = k_desc0 + (static_cast<uint64_t>((k % KS) * Plan::kTileBytes) >> 4);
-        const uint32_t d_tmem = tmem_base + kColS + (k & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
-          tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        tc::commit(bar_s_full + 8 * (k & 1));
-        tc::commit(bar_k_empty + 8 * (k % KS));
-      };
-      // Q is staged into TMEM by the softmax warps while the first K/V tiles
-      // are in flight
-      bool ok = tc_wait(bar_q_ready, 0, abort_flag) && tc_wait(bar_k_full, 0, abort_flag);
-      if (ok) {
-        tc::fence_after_sync();
-        issue_qk(0);
-      }
+      bool ok = true;
       for (int k = 0; ok && k < my_tiles; ++k) {
-        if (k + 1 < my_tiles) {
-          // the S/P buffer of tile k+1 last held P(k-1), read by PV(k-1),
-          // which was issued earlier and runs first
-          ok = tc_wait(bar_k_full + 8 * ((k + 1) % KS), ((k + 1) / KS) & 1, abort_flag);
-          if (!ok) break;
-          tc::fence_after_sync();
-          issue_qk(k + 1);
-        }
         ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag) &&
              tc_wait(bar_v_ready + 8 * (k % VS), (k / VS) & 1, abort_flag);
         if (!ok) break;
@@ -343,13 +320,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc::commit(bar_v_empty + 8 * (k % VS));
         tc::commit(bar_o_done);
+        tc::commit(bar_pv_done + 8 * (k & 1));
       }
       if (!ok) {
         if (*abort_flag == 0) set_status(a.status, kDevTimeout);
         *abort_flag = 1;
       }
-      // wait (bounded) until every MMA issued here has completed, so the
-      // tensor memory is never freed under a running MMA
+      // mma_final completes when both issuing lanes' MMAs have all completed
+      tc::commit(bar_final);
+      if (!ptx::mbar_wait(bar_final, 0)) set_status(a.status, kDevTimeout);
+    }
+    return;
+  }
+
+  // =================================================================== QK issuer
+  if (warp == 1) {
+    if (lane == 0 && my_tiles > 0) {
+      // M = 64: the rows never exceed 64, and an M=64 MMA costs the same
+      // issue time as M=128 for half the tensor work (and power)
+      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(64, 64, 0, 0);    // A (Q, TMEM), B (K) K-major
+      // descriptor start addresses are in 16-byte units in the low bits, so
+      // moving an operand by n bytes adds n >> 4 to the descriptor
+      const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
+      // Q is staged into TMEM by the softmax warps while the first K/V tiles
+      // are in flight
+      bool ok = tc_wait(bar_q_ready, 0, abort_flag);
+      for (int k = 0; ok && k < my_tiles; ++k) {
+        // S/P buffer k & 1 last held P(k-2): PV(k-2), issued by the other
+        // lane, must have completed (its phase of pv_done; the next phase
+        // needs P(k), which needs this S)
+        if (k >= 2 && !(ok = tc_wait(bar_pv_done + 8 * (k & 1), ((k - 2) >> 1) & 1, abort_flag))) break;
+        if (!(ok = tc_wait(bar_k_full + 8 * (k % KS), (k / KS) & 1, abort_flag))) break;
+        tc::fence_after_sync();
+        const uint64_t kd = k_desc0 + (static_cast<uint64_t>((k % KS) * Plan::kTileBytes) >> 4);
+        const uint32_t d_tmem = tmem_base + kColS + (k & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
+          tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(bar_s_full + 8 * (k & 1));
+        tc::commit(bar_k_empty + 8 * (k % KS));
+      }
+      if (!ok) {
+        if (*abort_flag == 0) set_status(a.status, kDevTimeout);
+        *abort_flag = 1;
+      }
+      // wait (bounded) until every MMA of both issuing lanes has completed,
+      // so the tensor memory is never freed under a running MMA
       tc::commit(bar_final);
       if (!ptx::mbar_wait(bar_final, 0)) set_status(a.status, kDevTimeout);
     }
