@@ -471,10 +471,10 @@ def cores_used():
 # hashes to the value it was captured on, and only for that workload.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "de533333a847358c9f82325a5a119c0ee4141083d75920283861a55c13863767",
+    "sha256": "5f33eae70ca830cbddf5bf4dfba5067452c6ca71ac59ecd5c8d27d8c76f13476",
     "workload": "1m: batch 1, 16q/2kv heads, D=256, page 64, ctx 1048576, S=4, W=4096, gamma=3, 10 verify layers",
-    # mean of two captured launches: 2,147,901,440 + 5,658,368 and 2,147,835,136 + 195,328 bytes
-    "bytes": 2150795136,
+    # mean of two captured launches: 2,147,834,112 + 3,779,328 and 2,148,131,328 + 800,000 bytes
+    "bytes": 2150272384,
 }
 
 
