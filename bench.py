@@ -467,11 +467,12 @@ def cores_used():
 
 # DRAM traffic of one verify_tc_kernel launch (dram__bytes_read.sum +
 # dram__bytes_write.sum) from one ncu capture of this script on the default
-# workload.  It is reported as roofline.traffic only while the kernel source
-# hashes to the value it was captured on, and only for that workload.
+# workload.  It is reported as roofline.traffic only while the kernel's code
+# (its sources with comments and whitespace removed) hashes to the value it
+# was captured on, and only for that workload.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "5f33eae70ca830cbddf5bf4dfba5067452c6ca71ac59ecd5c8d27d8c76f13476",
+    "sha256": "e411d45f0fce0021a163c5d084eb44c026751852141000aa997f89913551ee9f",
     "workload": "1m: batch 1, 16q/2kv heads, D=256, page 64, ctx 1048576, S=4, W=4096, gamma=3, 10 verify layers",
     # mean of two captured launches: 2,147,834,112 + 3,779,328 and 2,148,131,328 + 800,000 bytes
     "bytes": 2150272384,
@@ -482,10 +483,13 @@ def verify_traffic(desc: str):
     import hashlib
     if VERIFY_TRAFFIC["bytes"] is None or desc != VERIFY_TRAFFIC["workload"]:
         return None
+    import re
     h = hashlib.sha256()
     for rel in VERIFY_TRAFFIC["sources"]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            code = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+        code = re.sub(r"//[^\n]*", "", code)
+        h.update(" ".join(code.split()).encode())
     return VERIFY_TRAFFIC["bytes"] if h.hexdigest() == VERIFY_TRAFFIC["sha256"] else None
 
 

@@ -18,33 +18,38 @@
 // 16 (r % 4) + r / 4), so the rows spread over the four lane quadrants and
 // each softmax warp owns a quarter of them.
 //
-// Roles: warp 0 streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
-// into two shared-memory rings (KS and VS tiles deep) with TMA, one lane per ring: a K
-// tile is released as soon as its S = Q K^T has completed, a V tile only
-// after its O += P V, so K loads run ahead of the softmax instead of waiting
-// for the slower PV of the same tile; warp 1 allocates the tensor
-// memory and one lane issues S = Q K^T (M=64, N=64, K from shared memory,
-// K-major) while one lane of warp 10 issues O += P V (M=64, N=256, V read
-// MN-major straight from the TMA tile): a lane issues a small tcgen05.mma
-// only every ~66 cycles, so two issuing lanes keep the tensor pipe busier; warps 2..5 run the softmax, one thread per
-// row: the row's scores come out of TMEM, the maximum and sum are taken
-// inside the thread, and P goes back into TMEM in fp16; warps 6..9 convert
-// each landed V tile in place from bf16 to fp16 (and zero its rows past the
-// sequence end).  The value product is therefore fp16 x fp16 -> fp32: P
-// carries a relative rounding of at most 2^-11 (bf16 would give 2^-8 and miss
-// a 1e-3 relative-L2 bound), and V is exact for every |v| < 2^16 (below 2^-17
-// the absolute error stays under 2^-25); a larger |v| saturates and raises
-// WMTP_DEV_V_RANGE.  On sm_100 a tcgen05.mma of these shapes costs a fixed
-// ~100 cycles, so one fp16 MMA per 16 tokens instead of a bf16 hi + lo pair
-// is what keeps the block under the HBM time of a tile.
+// Roles:
+//   warp 0     streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
+//              into two shared-memory rings (KS and VS tiles deep) with TMA,
+//              one lane per ring; a K tile is released as soon as its
+//              S = Q K^T has completed, a V tile only after its O += P V, so K
+//              loads run ahead of the softmax;
+//   warp 1     allocates the tensor memory; one lane issues S = Q K^T (M=64,
+//              N=64, K from shared memory, K-major);
+//   warp 10    one lane issues O += P V (M=64, N=256, V read MN-major straight
+//              from the TMA tile).  A lane issues a small tcgen05.mma only
+//              every ~66 cycles, so the two streams issue from two lanes;
+//   warps 2-5  stage Q into TMEM, then run the softmax, one thread per row:
+//              the row's scores come out of TMEM, the maximum and sum are
+//              taken inside the thread, and P goes back into TMEM in fp16;
+//   warps 6-9  convert each landed V tile in place from bf16 to fp16 (and
+//              zero its rows past the sequence end).
+// The value product is therefore fp16 x fp16 -> fp32: P carries a relative
+// rounding of at most 2^-11 (bf16 would give 2^-8 and miss a 1e-3 relative-L2
+// bound), and V is exact for every |v| < 2^16 (below 2^-17 the absolute error
+// stays under 2^-25); a larger |v| saturates and raises WMTP_DEV_V_RANGE.  One
+// fp16 MMA per 16 tokens (an N=256 MMA keeps the tensor pipe ~134 cycles)
+// instead of a bf16 hi + lo pair is what keeps PV well under the HBM time of
+// a tile.
 // The reference maximum of a row is raised only when the tile maximum
 // exceeds it by more than 2^8 (weights then stay below 256, well inside
 // fp16), and only then is that row of O rescaled in TMEM, after the previous
 // PV completed.
 //
 // Every mbarrier wait is bounded; a wait that gives up raises
-// WMTP_DEV_TIMEOUT, stops the pipeline, waits (bounded) for the MMAs already
-// issued and frees the tensor memory before the CTA exits.
+// WMTP_DEV_TIMEOUT and stops the pipeline; the producers still wait (bounded)
+// for their copies in flight and the issuing lanes for their MMAs, and the
+// tensor memory is freed before the CTA exits.
 #pragma once
 
 #include <cuda.h>
