@@ -1,14 +1,19 @@
 // Split-KV decode attention for Windowed-MTP draft and verify steps (sm_100a).
 //
-// One kernel template serves the three attention calls of a decode step:
+// One kernel template serves the attention calls of a decode step:
 //   * native draft  : 1 query x G heads over the draft layer's paged cache
 //                     ("Windowed-MTP ..." arxivlens view, Abstract: the draft
 //                     head reads the full KV cache in each draft forward);
 //   * windowed draft: the same query over the compact sink + window ring
-//                     (same Abstract; readpriors post, What happened);
+//                     (same Abstract; readpriors post, What happened), or
+//                     over the sink + window positions of the paged cache
+//                     (paged_window: only the tiles holding those positions
+//                     are loaded);
 //   * verify        : gamma+1 causal queries x G heads over a target layer's
 //                     paged cache (same Abstract: verification stays
-//                     full-context).
+//                     full-context) for blocks outside the tcgen05 verify
+//                     kernel's range (head_dim 64, or 8 or fewer rows); with
+//                     q_pos0 the cache may hold a slice of a longer context.
 //
 // Work decomposition: CTA = (split, kv head, sequence).  All query rows that
 // share the KV head (rows = num_q * G, padded to NT*8) are processed together,
@@ -30,7 +35,9 @@
 //   4. O^T += V^T P^T on tensor cores, warp w owning head-dim columns
 //      [w*D/4, (w+1)*D/4).
 // At the end each CTA writes its split's fp32 partial output and log-sum-exp;
-// a combine kernel merges the splits.
+// a combine kernel merges the splits.  The kernel is launched as a
+// programmatic dependent: barrier set-up runs before griddepcontrol.wait,
+// every global-memory access after it.
 //
 // Masking is by selection (score := -inf), never by multiplication, and V rows
 // past the valid length are zeroed in shared memory, so stale or non-finite
