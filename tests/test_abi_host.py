@@ -134,3 +134,24 @@ def test_python_binding_raises_on_wrong_tensors():
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         L.load(str(tmp_path / "missing.so"))
+
+
+def test_windowed_paged_and_slice_reject_bad_args(lib):
+    desc = L.PagedKVDesc(None, None, 8, None, 8, None)
+    size = c_size_t(0)
+    # the windowed-over-pages draft needs window >= 1 and sinks >= 0
+    for kw in (dict(window=0), dict(sinks=-1)):
+        assert lib.wmtp_draft_attn_windowed_paged(byref(_p(**kw)), 1, None, byref(desc), None, 1, None, None,
+                                                  byref(size), None, None) == L.WMTP_ERR_INVALID_ARG
+    assert lib.wmtp_draft_attn_windowed_paged(byref(_p(num_heads_q=15)), 1, None, byref(desc), None, 1, None,
+                                              None, byref(size), None, None) == L.WMTP_ERR_INVALID_ARG
+    assert lib.wmtp_draft_attn_windowed_paged(byref(_p()), 0, None, byref(desc), None, 1, None, None,
+                                              byref(size), None, None) == 0  # empty batch: size query only
+    # a slice verify with a workspace needs the query positions
+    ws = ctypes.create_string_buffer(512)
+    have = c_size_t(256)
+    assert lib.wmtp_verify_attn_slice(byref(_p()), 1, 4, None, byref(desc), None, None, 1, None,
+                                      ctypes.addressof(ws) // 256 * 256 + 256, byref(have), None,
+                                      None) == L.WMTP_ERR_INVALID_ARG
+    assert lib.wmtp_verify_attn_slice(byref(_p()), 1, 9, None, byref(desc), None, None, 1, None, None,
+                                      byref(size), None, None) == L.WMTP_ERR_UNSUPPORTED  # 72 rows
