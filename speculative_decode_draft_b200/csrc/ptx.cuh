@@ -82,9 +82,9 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
-// 3-D tiled TMA load into this CTA's shared memory, completing on `bar`.
-// No cluster multicast.  x (the innermost coordinate) must be a multiple of
-// 8 bf16 elements (16 bytes); callers pass multiples of 64.
+// 3-D tiled TMA load into this CTA's own shared memory (no other CTA is
+// written), completing on `bar`.  x (the innermost coordinate) must be a
+// multiple of 8 bf16 elements (16 bytes); callers pass multiples of 64.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x,
                                             int y, int z, uint64_t policy) {
   asm volatile(
