@@ -318,6 +318,29 @@ wmtp_status wmtp_draft_attn_full_noalloc(const wmtp_params* params, int32_t batc
                                          const wmtp_paged_kv* kv, void* out, int32_t out_fp32,
                                          float* lse_out, int32_t* status_word, void* stream);
 
+/*
+ * wmtp_selftest_wait -- run the bounded in-kernel wait on its own.
+ * The paper has no counterpart to this call, and it is not on the attention
+ * path.  It lets a test check on a live GPU that a wait which never completes
+ * gives up, reports WMTP_DEV_TIMEOUT, and leaves the context usable.
+ *
+ * One thread initialises a shared-memory mbarrier that expects one arrival.
+ * It then waits for the barrier's first phase, with the same bounded wait
+ * every attention kernel uses: it gives up after WMTP_WAIT_LIMIT_CYCLES SM
+ * clocks, about 2 s at 1.9 GHz.
+ *   arrive != 0 : the thread arrives first, so the wait returns at once and
+ *                 no bit is set.
+ *   arrive == 0 : nothing arrives.  The wait gives up at the limit and
+ *                 WMTP_DEV_TIMEOUT is OR-ed into *status_word.
+ *   status_word : device int32, NULL = skip.
+ *   cycles_out  : device int64, NULL = skip.  Receives the SM clocks the wait
+ *                 took.
+ * A misaligned pointer returns WMTP_ERR_INVALID_ARG; a failed launch returns
+ * WMTP_ERR_CUDA.  Asynchronous on `stream` like every other call.
+ */
+#define WMTP_WAIT_LIMIT_CYCLES 4000000000LL
+wmtp_status wmtp_selftest_wait(int32_t arrive, int32_t* status_word, int64_t* cycles_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,6 +20,7 @@ from .api import (  # noqa: F401
     plan_admission,
     ring_append,
     ring_reset,
+    selftest_wait,
     splitkv_combine,
     verify_attn,
     workspace_bytes,

@@ -26,6 +26,7 @@ DEV_RING_STATE = 0x4
 DEV_UNDO_FULL = 0x8
 DEV_TIMEOUT = 0x10
 DEV_V_RANGE = 0x20
+WAIT_LIMIT_CYCLES = 4000000000  # WMTP_WAIT_LIMIT_CYCLES
 
 EXPORTS = (
     "wmtp_status_string",
@@ -46,6 +47,7 @@ EXPORTS = (
     "wmtp_pool_alloc",
     "wmtp_pool_release",
     "wmtp_plan_admission",
+    "wmtp_selftest_wait",
 )
 
 # Size of the fixed scratch array behind wmtp_draft_attn_full_noalloc.
@@ -172,6 +174,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.wmtp_plan_admission.restype = c_int32
     lib.wmtp_plan_admission.argtypes = [PP, ctypes.c_int64, c_int32, c_int32, c_int32, ctypes.c_int64,
                                         POINTER(Admission)]
+    lib.wmtp_selftest_wait.restype = c_int32
+    lib.wmtp_selftest_wait.argtypes = [c_int32, c_void_p, c_void_p, c_void_p]
     if path is None:
         _lib = lib
     return lib

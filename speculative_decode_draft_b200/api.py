@@ -302,6 +302,19 @@ def new_status(device) -> torch.Tensor:
     return torch.zeros(1, dtype=I32, device=device)
 
 
+def selftest_wait(arrive: bool, *, status=None, cycles=None, stream=None) -> None:
+    """One bounded in-kernel wait (``wmtp_selftest_wait``).  Without ``arrive``
+    nothing completes the barrier: the wait gives up after
+    ``WAIT_LIMIT_CYCLES`` SM clocks and sets ``DEV_TIMEOUT`` in ``status``.
+    ``cycles`` (int64 ``[1]``) receives the clocks the wait took."""
+    if status is not None:
+        _need(status, I32, "status")
+    if cycles is not None:
+        _need(cycles, torch.int64, "cycles")
+    L.check("wmtp_selftest_wait", L.load().wmtp_selftest_wait(
+        int(bool(arrive)), _ptr(status), _ptr(cycles), _stream(stream)))
+
+
 # ---------------------------------------------------------------- serving-side helpers (host only)
 class PagePool:
     """Free-list allocator over the page indices of one pool tensor

@@ -18,7 +18,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libwmtp.so")
-SOURCES = [os.path.join(HERE, "csrc", "wmtp_abi.cu"), os.path.join(HERE, "csrc", "page_pool.cpp")]
+SOURCES = [os.path.join(HERE, "csrc", "wmtp_abi.cu"), os.path.join(HERE, "csrc", "page_pool.cpp"),
+           os.path.join(HERE, "csrc", "selftest.cu")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -155,3 +155,10 @@ def test_windowed_paged_and_slice_reject_bad_args(lib):
                                       None) == L.WMTP_ERR_INVALID_ARG
     assert lib.wmtp_verify_attn_slice(byref(_p()), 1, 9, None, byref(desc), None, None, 1, None, None,
                                       byref(size), None, None) == L.WMTP_ERR_UNSUPPORTED  # 72 rows
+
+
+def test_selftest_wait_rejects_misaligned_pointers(lib):
+    # checked before anything is launched, so this runs without a GPU
+    assert lib.wmtp_selftest_wait(0, None, 4, None) == L.WMTP_ERR_INVALID_ARG
+    assert lib.wmtp_selftest_wait(0, 2, None, None) == L.WMTP_ERR_INVALID_ARG
+    assert L.WAIT_LIMIT_CYCLES == 4_000_000_000
