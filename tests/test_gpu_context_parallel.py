@@ -17,7 +17,7 @@ import synth
 import speculative_decode_draft_b200 as w
 from speculative_decode_draft_b200.context_parallel import slice_query_positions
 
-from _helpers import assert_close, assert_lse_close, cache_of, f64
+from _helpers import assert_close, assert_lse_close, f64
 
 pytestmark = pytest.mark.gpu
 

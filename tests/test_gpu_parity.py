@@ -14,7 +14,7 @@ import synth
 import speculative_decode_draft_b200 as w
 from speculative_decode_draft_b200 import _lib as L
 
-from _helpers import (assert_close, assert_lse_close, bits, bf16_ulp_diff, cache_of, dense_kv_f64, f64)
+from _helpers import (assert_close, assert_lse_close, bits, bf16_ulp_diff, cache_of, f64)
 
 pytestmark = pytest.mark.gpu
 

@@ -12,7 +12,6 @@ here leaves every other test already run.
 
 from ctypes import byref, c_size_t, c_void_p
 
-import numpy as np
 import pytest
 import torch
 
