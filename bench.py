@@ -60,6 +60,11 @@ def parse(argv=None):
                     help="context x gamma x window sweep of native/windowed step time (one JSON line per point)")
     ap.add_argument("--eager", action="store_true",
                     help="time the steps as eager launches instead of one CUDA graph per decode step")
+    ap.add_argument("--admission", action="store_true",
+                    help="admit 1M-context requests into one fixed KV budget through the page allocator, "
+                         "native vs windowed, then decode each arm's admitted batch (one JSON line)")
+    ap.add_argument("--kv-budget-gb", type=float, default=130.0,
+                    help="KV budget of --admission in GB (1e9 bytes)")
     return ap.parse_args(argv)
 
 
@@ -218,9 +223,15 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 class Workload:
     """All device state of one replica: verify layers, the draft pool, the
-    ring, and per-step inputs for warmup + timed steps."""
+    ring, and per-step inputs for warmup + timed steps.
 
-    def __init__(self, args, rank, device):
+    ``kv`` (optional) builds the paged caches instead of one seeded pool per
+    layer: ``kv(workload, capacity_tokens) -> (verify caches, draft cache or
+    None)``; without a draft cache the ring is filled with seeded tokens and
+    only the windowed arm can run.  ``batch`` overrides the workload's batch
+    (every sequence then has the same context)."""
+
+    def __init__(self, args, rank, device, kv=None, batch=None):
         import numpy as np
         import torch
 
@@ -231,7 +242,7 @@ class Workload:
         self.torch = torch
         base = synth.workload(args.config)
         self.wl = base
-        self.B = base.batch
+        self.B = batch if batch is not None else base.batch
         self.Hq, self.Hkv, self.D, self.P = base.num_heads_q, base.num_heads_kv, base.head_dim, base.page_size
         self.G = self.Hq // self.Hkv
         self.S = base.sinks
@@ -241,6 +252,8 @@ class Workload:
         self.steps_total = args.steps + args.warmup
         # committed context per sequence at the first step (ragged4: one per sequence)
         self.n0s = [int(args.ctx)] * base.batch if args.ctx else [int(c) for c in base.context]
+        if batch is not None:
+            self.n0s = [max(self.n0s)] * batch
         self.n0 = max(self.n0s)
         seed = base.seed + 1000 * rank
         self.seed = seed
@@ -258,15 +271,20 @@ class Workload:
                           gamma_max=self.gamma)
         kvs = base.kv_scale
         shuf = base.shuffle_pages
-        # verify layers: independent random KV, n0 committed tokens each
-        self.layers = [synth.paged_kv(seed + 10 + l, self.B, self.Hkv, self.D, self.P, self.n0s,
-                                      cap, kvs, shuf, device=dev) for l in range(self.L)]
-        # the draft layer's own KV (native arm reads it in full)
-        self.draft = synth.paged_kv(seed + 5, self.B, self.Hkv, self.D, self.P, self.n0s, cap, kvs,
-                                    shuf, device=dev)
-        self.caches = [w.PagedCache(k.k_pool, k.v_pool, k.page_table, k.kv_len) for k in self.layers]
-        self.draft_cache = w.PagedCache(self.draft.k_pool, self.draft.v_pool, self.draft.page_table,
-                                        self.draft.kv_len)
+        self.draft = None
+        if kv is None:
+            # verify layers: independent random KV, n0 committed tokens each
+            layers = [synth.paged_kv(seed + 10 + l, self.B, self.Hkv, self.D, self.P, self.n0s,
+                                     cap, kvs, shuf, device=dev) for l in range(self.L)]
+            # the draft layer's own KV (native arm reads it in full)
+            self.draft = synth.paged_kv(seed + 5, self.B, self.Hkv, self.D, self.P, self.n0s, cap, kvs,
+                                        shuf, device=dev)
+            self.caches = [w.PagedCache(k.k_pool, k.v_pool, k.page_table, k.kv_len) for k in layers]
+            self.draft_cache = w.PagedCache(self.draft.k_pool, self.draft.v_pool, self.draft.page_table,
+                                            self.draft.kv_len)
+            del layers
+        else:
+            self.caches, self.draft_cache = kv(self, cap)
         # per-step inputs
         T = self.steps_total
         g = torch.Generator(device=dev)
@@ -300,22 +318,29 @@ class Workload:
         self.l_draft = torch.empty(self.B, self.Hq, **f32)
         self.o_ver = torch.empty(self.B, self.gamma + 1, self.Hq, self.D, **f32)
         self.l_ver = torch.empty(self.B, self.gamma + 1, self.Hq, **f32)
-        # ring of the windowed arm, filled from the draft layer's history
+        # ring of the windowed arm, filled from the draft layer's history (or
+        # with seeded tokens when there is no paged draft layer)
         self.ring = w.Ring.allocate(self.p, self.B, dev)
-        kd = torch.zeros(self.B, self.n0, self.Hkv, self.D, dtype=torch.bfloat16, device=dev)
-        vd = torch.zeros_like(kd)
-        for b in range(self.B):
-            k, v = synth.dense_from_paged(self.draft, b, self.n0s[b])
-            kd[b, :self.n0s[b]].copy_(k)
-            vd[b, :self.n0s[b]].copy_(v)
-        w.ring_append(self.p, self.ring, kd, vd, torch.tensor(self.n0s, **i32), status=self.status)
-        del kd, vd
+        if self.draft is not None:
+            kd = torch.zeros(self.B, self.n0, self.Hkv, self.D, dtype=torch.bfloat16, device=dev)
+            vd = torch.zeros_like(kd)
+            for b in range(self.B):
+                k, v = synth.dense_from_paged(self.draft, b, self.n0s[b])
+                kd[b, :self.n0s[b]].copy_(k)
+                vd[b, :self.n0s[b]].copy_(v)
+            w.ring_append(self.p, self.ring, kd, vd, torch.tensor(self.n0s, **i32), status=self.status)
+            del kd, vd
+        else:
+            from speculative_decode_draft_b200.timing import fill_ring_to
+            fill_ring_to(self.p, self.ring, self.n0, seed + 6, dev)
         torch.cuda.synchronize()
+        ver_pages = self.caches[0].page_table.shape[1]
+        draft_pages = self.draft_cache.page_table.shape[1] if self.draft_cache is not None else 1
         self.workspace = torch.empty(max(
-            w.workspace_bytes("full", self.p, self.B, max_pages=self.draft.max_pages),
-            w.workspace_bytes("verify", self.p, self.B, num_q=self.gamma + 1, max_pages=self.layers[0].max_pages),
+            w.workspace_bytes("full", self.p, self.B, max_pages=draft_pages),
+            w.workspace_bytes("verify", self.p, self.B, num_q=self.gamma + 1, max_pages=ver_pages),
             w.workspace_bytes("windowed", self.p, self.B),
-            w.workspace_bytes("windowed_paged", self.p, self.B, max_pages=self.draft.max_pages)),
+            w.workspace_bytes("windowed_paged", self.p, self.B, max_pages=draft_pages)),
             dtype=torch.uint8, device=dev)
 
     # -- kernel launches of one step (for gpu_launches)
@@ -325,55 +350,67 @@ class Workload:
         return self.gamma * (1 + 2) + self.L * (1 + 2)
 
     # -- one decode step; `ev` collects (kind, start_event, end_event)
-    def step(self, s: int, arm: str, ev=None, inputs=None, external_events: bool = False):
+    # names of the per-step input tensors (first dimension: the step)
+    STEP_INPUTS = ("q_draft", "k_draft", "v_draft", "k_bonus", "v_bonus", "q_ver", "k_ver", "v_ver",
+                   "len_draft", "pos_draft", "len_ver", "pos_ver", "trunc_to", "n_bonus")
+
+    def step_inputs(self, s: int) -> dict:
+        """This step's inputs: queries, new K/V, lengths and positions, the
+        rollback targets and bonus-token counts drawn from the acceptance."""
+        return {name: getattr(self, name)[s] for name in self.STEP_INPUTS}
+
+    def step(self, s: int, arm: str, ev=None, inputs=None, external_events: bool = False, outputs=None):
+        """One decode step.  ``inputs`` (a dict like ``step_inputs``) replaces
+        the resident inputs of step ``s``; ``outputs`` (``{"draft": [gamma,
+        ...], "verify": [L, ...]}``, e.g. pinned host buffers) receives every
+        attention output of the step."""
         torch, w = self.torch, self.w
 
         def E(**kw):  # events inside a captured graph must be graph nodes
             return torch.cuda.Event(external=external_events, **kw)
-        qd = self.q_draft[s] if inputs is None else inputs["q_draft"]
-        qv = self.q_ver[s] if inputs is None else inputs["q_ver"]
+        x = inputs if inputs is not None else self.step_inputs(s)
         for j in range(self.gamma):
             if arm == "windowed":
-                w.ring_append(self.p, self.ring, self.k_draft[s, j], self.v_draft[s, j], self.one,
+                w.ring_append(self.p, self.ring, x["k_draft"][j], x["v_draft"][j], self.one,
                               speculative=True, status=self.status)
                 a = E(enable_timing=True) if ev is not None else None
                 if a is not None:
                     a.record()
-                w.draft_attn_windowed(self.p, qd[j], self.ring, out=self.o_draft, lse=self.l_draft,
+                w.draft_attn_windowed(self.p, x["q_draft"][j], self.ring, out=self.o_draft, lse=self.l_draft,
                                       workspace=self.workspace, status=self.status)
             else:
-                self.draft_cache.kv_len = self.len_draft[s, j]
-                w.paged_write(self.p, self.draft_cache, self.pos_draft[s, j], self.k_draft[s, j],
-                              self.v_draft[s, j], status=self.status)
+                self.draft_cache.kv_len = x["len_draft"][j]
+                w.paged_write(self.p, self.draft_cache, x["pos_draft"][j], x["k_draft"][j], x["v_draft"][j],
+                              status=self.status)
                 a = E(enable_timing=True) if ev is not None else None
                 if a is not None:
                     a.record()
-                w.draft_attn_full(self.p, qd[j], self.draft_cache, out=self.o_draft, lse=self.l_draft,
+                w.draft_attn_full(self.p, x["q_draft"][j], self.draft_cache, out=self.o_draft, lse=self.l_draft,
                                   workspace=self.workspace, status=self.status)
             if ev is not None:
                 bnd = E(enable_timing=True)
                 bnd.record()
                 ev.append(("draft", a, bnd))
-            if inputs is not None:
-                inputs["out_draft"][j].copy_(self.o_draft, non_blocking=True)
+            if outputs is not None:
+                outputs["draft"][j].copy_(self.o_draft, non_blocking=True)
         for l in range(self.L):
             c = self.caches[l]
-            c.kv_len = self.len_ver[s]
-            w.paged_write(self.p, c, self.pos_ver[s], self.k_ver[s, l], self.v_ver[s, l], status=self.status)
+            c.kv_len = x["len_ver"]
+            w.paged_write(self.p, c, x["pos_ver"], x["k_ver"][l], x["v_ver"][l], status=self.status)
             a = E(enable_timing=True) if ev is not None else None
             if a is not None:
                 a.record()
-            w.verify_attn(self.p, qv[l], c, out=self.o_ver, lse=self.l_ver, workspace=self.workspace,
+            w.verify_attn(self.p, x["q_ver"][l], c, out=self.o_ver, lse=self.l_ver, workspace=self.workspace,
                           status=self.status)
             if ev is not None:
                 bnd = E(enable_timing=True)
                 bnd.record()
                 ev.append(("verify", a, bnd))
-            if inputs is not None:
-                inputs["out_ver"][l].copy_(self.o_ver, non_blocking=True)
+            if outputs is not None:
+                outputs["verify"][l].copy_(self.o_ver, non_blocking=True)
         if arm == "windowed":
-            w.ring_append(self.p, self.ring, self.k_bonus[s], self.v_bonus[s], self.n_bonus[s],
-                          truncate_to=self.trunc_to[s], status=self.status)
+            w.ring_append(self.p, self.ring, x["k_bonus"], x["v_bonus"], x["n_bonus"],
+                          truncate_to=x["trunc_to"], status=self.status)
 
     def snapshot_ring(self):
         r = self.ring
@@ -405,53 +442,120 @@ def algorithmic_bytes(wl, kind: str, ctxs) -> float:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (baseline, not target)
 # ---------------------------------------------------------------------------
-def oracle_step_model(args, sample_ctx: int, repeats: int = 1):
-    """Time the fp64 oracle on one sample of each unit at `sample_ctx` tokens
-    (the fastest of `repeats` runs of each), return modelled microseconds per
-    decode step at the workload's context."""
-    import numpy as np
+ORACLE_CHUNK = 65536  # tokens per chunk of the oracle's full-context units
 
-    import oracle
-    import synth
-    base = synth.workload(args.config)
-    Hq, Hkv, D, P, S = base.num_heads_q, base.num_heads_kv, base.head_dim, base.page_size, base.sinks
-    W = args.window if args.config in ("1m", "128k") else base.window
-    gamma = args.gamma
-    L = args.layers if args.layers is not None else base.verify_layers
-    ctxs = [int(args.ctx)] * base.batch if args.ctx else [int(c) for c in base.context]
-    n = min(sample_ctx, max(ctxs))
-    kv = synth.paged_kv(base.seed, 1, Hkv, D, P, [n + gamma + 1], n + gamma + 1 + P, base.kv_scale,
-                        base.shuffle_pages, device="cpu")
-    kp = kv.k_pool.double().numpy()
-    vp = kv.v_pool.double().numpy()
-    pt = kv.page_table.numpy()
-    q1 = synth.queries(7, (1, Hq, D)).double().numpy()
-    qv = synth.queries(8, (1, gamma + 1, Hq, D)).double().numpy()
-    scale = 1 / math.sqrt(D)
-    t_draft = t_ver = math.inf
-    work = 0.0
-    for _ in range(repeats):
-        t0 = time.perf_counter()
-        oracle.draft_attn_full(q1, kp, vp, pt, np.array([n + 1]), P, scale)
-        t1 = time.perf_counter()
-        oracle.verify_attn(qv, kp, vp, pt, np.array([n + gamma + 1]), P, scale)
-        t2 = time.perf_counter()
-        t_draft, t_ver = min(t_draft, t1 - t0), min(t_ver, t2 - t1)
-        work += t2 - t0
-    # windowed: the ring holds S+W entries whatever the context
-    ring = oracle.RingModel(S, W, gamma, Hkv, D, dtype=np.float64)
-    m = min(n, S + W)
-    hist_k = np.stack([kp[pt[0, p // P], :, p % P] for p in range(m)])
-    hist_v = np.stack([vp[pt[0, p // P], :, p % P] for p in range(m)])
-    ring.call(-1, hist_k, hist_v, False)
-    t0 = time.perf_counter()
-    oracle.draft_attn_windowed(q1, [ring], scale)
-    t_win = time.perf_counter() - t0
-    f = sum(ctxs) / n  # every sequence's attention scales with its own context
-    native_us = (gamma * t_draft * f + L * t_ver * f) * 1e6
-    windowed_us = (gamma * t_win * len(ctxs) + L * t_ver * f) * 1e6
-    return {"native_us": native_us, "windowed_us": windowed_us, "sample_ctx": n, "work_s": work + t_win,
-            "t_draft_s": t_draft, "t_verify_s": t_ver, "t_windowed_s": t_win}
+
+class OracleUnits:
+    """The fp64 oracle timed on one unit of each kind at the workload's full
+    context: one verify layer (gamma+1 causal queries), one native draft (one
+    query over the whole cache) and one windowed draft (one query over S + W
+    ring entries), every KV head, sequence 0 of the workload.
+
+    The context is processed in 64K-token chunks: per chunk and KV head one
+    ``oracle.attend_prefixes`` call (all query rows of the head, each with its
+    causal limit inside the chunk), then ``oracle.splitkv_combine`` over the
+    chunks -- both oracle functions, pinned by the oracle's tests.  Only the
+    oracle calls are timed; drawing the seeded bf16 K/V and widening each
+    chunk to fp64 are not.  A decode step is modelled from the measured units
+    as gamma x draft + L x verify (windowed or native draft)."""
+
+    def __init__(self, args):
+        import torch
+
+        import synth
+        base = synth.workload(args.config)
+        self.Hq, self.Hkv, self.D = base.num_heads_q, base.num_heads_kv, base.head_dim
+        self.G = self.Hq // self.Hkv
+        self.S = base.sinks
+        self.W = args.window if args.config in ("1m", "128k") else base.window
+        self.gamma = args.gamma
+        self.L = args.layers if args.layers is not None else base.verify_layers
+        self.ctxs = [int(args.ctx)] * base.batch if args.ctx else [int(c) for c in base.context]
+        self.n = self.ctxs[0] + self.gamma + 1  # sequence 0, the verify block appended
+        self.scale = 1.0 / math.sqrt(self.D)
+        # seeded N(0, 1) values rounded to bf16 (numpy's generator: fast on the
+        # host for the 1M context), K/V of one layer kept as bf16
+        import numpy as np
+        rng = np.random.default_rng(base.seed + 4242)
+
+        def bf16(*shape):
+            return torch.from_numpy(rng.standard_normal(shape, dtype=np.float32)).to(torch.bfloat16)
+        self.k = bf16(self.n, self.Hkv, self.D)
+        self.v = bf16(self.n, self.Hkv, self.D)
+        self.qv = bf16(self.gamma + 1, self.Hq, self.D).double().numpy()
+        self.qd = bf16(self.Hq, self.D).double().numpy()
+        self._f64 = {}
+
+    def _chunk(self, c0, c1, kvh):
+        # widened once, then reused by every unit and step (8.6 GB of fp64 at 1M)
+        key = (c0, kvh)
+        if key not in self._f64:
+            self._f64[key] = (self.k[c0:c1, kvh].double().numpy(), self.v[c0:c1, kvh].double().numpy())
+        return self._f64[key]
+
+    def _full_context(self, qs_of, limits):
+        """attend_prefixes per chunk + splitkv_combine; returns timed seconds."""
+        import numpy as np
+
+        import oracle
+        t = 0.0
+        for kvh in range(self.Hkv):
+            qs = qs_of(kvh)
+            parts_o, parts_l = [], []
+            for c0 in range(0, self.n, ORACLE_CHUNK):
+                c1 = min(self.n, c0 + ORACLE_CHUNK)
+                K, V = self._chunk(c0, c1, kvh)
+                lengths = np.clip(np.asarray(limits) - c0, 0, c1 - c0)
+                t0 = time.perf_counter()
+                o, lse = oracle.attend_prefixes(qs, K, V, lengths, self.scale)
+                t += time.perf_counter() - t0
+                parts_o.append(o)
+                parts_l.append(lse)
+            t0 = time.perf_counter()
+            oracle.splitkv_combine(np.stack(parts_o, axis=1), np.stack(parts_l, axis=1))
+            t += time.perf_counter() - t0
+        return t
+
+    def verify_s(self):
+        G, Qn = self.G, self.gamma + 1
+        limits = [self.n - Qn + i + 1 for i in range(Qn) for _ in range(G)]  # row i * G + g: query i
+        return self._full_context(lambda kvh: self.qv[:, kvh * G:(kvh + 1) * G].reshape(Qn * G, self.D), limits)
+
+    def draft_native_s(self):
+        G = self.G
+        return self._full_context(lambda kvh: self.qd[kvh * G:(kvh + 1) * G], [self.n] * G)
+
+    def draft_windowed_s(self):
+        import numpy as np
+
+        import oracle
+        G = self.G
+        pos = oracle.window_positions(self.n, self.S, self.W)
+        t = 0.0
+        for kvh in range(self.Hkv):
+            K = self.k[pos, kvh].double().numpy()
+            V = self.v[pos, kvh].double().numpy()
+            t0 = time.perf_counter()
+            oracle.attend_prefixes(self.qd[kvh * G:(kvh + 1) * G], K, V, np.full(G, len(pos)), self.scale)
+            t += time.perf_counter() - t0
+        return t
+
+    def step_model(self):
+        """Measured unit times and the modelled decode step (us) of both arms;
+        every sequence of the workload costs its own context's share."""
+        tv, tn, tw = self.verify_s(), self.draft_native_s(), self.draft_windowed_s()
+        f = sum(self.ctxs) / self.ctxs[0]  # other sequences: same per-token cost at their own length
+        return {"verify_s": tv, "draft_native_s": tn, "draft_windowed_s": tw,
+                "native_us": (self.gamma * tn + self.L * tv) * f * 1e6,
+                "windowed_us": (self.gamma * tw * len(self.ctxs) + self.L * tv * f) * 1e6,
+                "work_s": tv + tn + tw}
+
+    def sample_desc(self):
+        return (f"fp64 numpy oracle, one verify layer ({self.gamma + 1} causal queries), one native draft and one "
+                f"windowed draft (S={self.S}, W={self.W}) at the full context of {self.n} tokens, every KV head "
+                f"({self.Hq}q/{self.Hkv}kv, D={self.D}), in {ORACLE_CHUNK}-token chunks (attend_prefixes per chunk, "
+                f"splitkv_combine); step modelled as gamma x draft + {self.L} x verify"
+                + ("" if len(self.ctxs) == 1 else f", scaled to the {len(self.ctxs)} sequences' contexts"))
 
 
 def cores_used():
@@ -466,31 +570,42 @@ def cores_used():
 
 
 # DRAM traffic of one verify_tc_kernel launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) from one ncu capture of this script on the default
-# workload.  It is reported as roofline.traffic only while the kernel's code
-# (its sources with comments and whitespace removed) hashes to the value it
-# was captured on, and only for that workload.
+# dram__bytes_write.sum) from one ncu capture on the 128K workload (a few GB
+# on the device), with the K/V tokens that launch read.  The traffic of a
+# launch grows in proportion to the tokens it reads (every K/V byte crosses
+# HBM once; the partials are a few MB), so it is scaled by tokens to the
+# bench's workload.  It is reported only while the kernel's code (its sources
+# with comments and whitespace removed) hashes to the value it was captured
+# on; otherwise roofline.traffic is null.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "e411d45f0fce0021a163c5d084eb44c026751852141000aa997f89913551ee9f",
-    "workload": "1m: batch 1, 16q/2kv heads, D=256, page 64, ctx 1048576, S=4, W=4096, gamma=3, 10 verify layers",
-    # mean of two captured launches: 2,147,834,112 + 3,779,328 and 2,148,131,328 + 800,000 bytes
-    "bytes": 2150272384,
+    "sha256": None,
+    "captured_on": None,
+    "tokens": None,   # K/V tokens read by the captured launch (per sequence, summed)
+    "bytes": None,
 }
 
 
-def verify_traffic(desc: str):
+def kernel_code_hash(root=None) -> str:
+    """sha256 of the verify kernel's sources with comments and whitespace removed."""
     import hashlib
-    if VERIFY_TRAFFIC["bytes"] is None or desc != VERIFY_TRAFFIC["workload"]:
-        return None
     import re
     h = hashlib.sha256()
     for rel in VERIFY_TRAFFIC["sources"]:
-        with open(os.path.join(ROOT, rel)) as f:
+        with open(os.path.join(root or ROOT, rel)) as f:
             code = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
         code = re.sub(r"//[^\n]*", "", code)
         h.update(" ".join(code.split()).encode())
-    return VERIFY_TRAFFIC["bytes"] if h.hexdigest() == VERIFY_TRAFFIC["sha256"] else None
+    return h.hexdigest()
+
+
+def verify_traffic(tokens: int):
+    """Captured DRAM bytes of one verify launch, scaled to a launch reading
+    `tokens` K/V tokens; None if nothing was captured for this kernel code."""
+    t = VERIFY_TRAFFIC
+    if t["bytes"] is None or not t["tokens"] or kernel_code_hash() != t["sha256"]:
+        return None
+    return t["bytes"] * tokens / t["tokens"]
 
 
 def workload_desc(args) -> str:
@@ -506,16 +621,18 @@ def workload_desc(args) -> str:
 
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle, timed on the host, per decode
-    step of the same workload (modelled from a bounded context sample)."""
+    """The reference arm: the fp64 CPU oracle on the host cores, per decode
+    step of the same workload (each step measures one verify layer, one native
+    draft and one windowed draft at the full context, and models the step from
+    them); rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
-    sample = 65536
+    units = OracleUnits(args)
     per = []
     for i in range(args.warmup + args.steps):
-        r = oracle_step_model(args, sample)
+        r = units.step_model()
         if i >= args.warmup:
             per.append(r)
     v = statistics.median(x["windowed_us"] for x in per)
@@ -524,10 +641,12 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(args),
-                   "native_us_per_step": statistics.median(x["native_us"] for x in per)},
+                   "native_us_per_step": statistics.median(x["native_us"] for x in per),
+                   "verify_s_per_layer": statistics.median(x["verify_s"] for x in per),
+                   "draft_native_s": statistics.median(x["draft_native_s"] for x in per),
+                   "draft_windowed_s": statistics.median(x["draft_windowed_s"] for x in per)},
         "cpu_baseline": {"value": v, "unit": "us/step", "cores": cores_used(), "kind": "oracle",
-                         "sample": f"one native draft, one windowed draft and one verify layer at {sample} "
-                                   "tokens per step, scaled linearly in context to the workload"},
+                         "sample": units.sample_desc()},
         "e2e": {"value": v, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -639,6 +758,131 @@ def run_sweep(args, rank: int, world: int, dev) -> int:
     return 0
 
 
+def time_single_arm(args, wk, arm: str, world: int) -> dict:
+    """Warm up one arm, capture each timed step as a CUDA graph, time K steps
+    between a barrier + synchronize on both sides (max over ranks)."""
+    import torch
+    for s in range(args.warmup):
+        wk.step(s, arm)
+    torch.cuda.synchronize()
+    graphs = []
+    for s in range(args.warmup, args.warmup + args.steps):
+        evs = []
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            wk.step(s, arm, ev=evs, external_events=True)
+        graphs.append((g, evs))
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for g, _ in graphs:
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    per = {}
+    for _, evs in graphs:
+        for kind, e0, e1 in evs:
+            per.setdefault(kind, []).append(e0.elapsed_time(e1) * 1000.0)
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    del graphs
+    return {"us_per_step": ms * 1000.0 / args.steps, "per_call_us": {k: statistics.mean(v) for k, v in per.items()}}
+
+
+def run_admission(args, rank: int, world: int, dev) -> int:
+    """The capacity side of Windowed-MTP (arxivlens view, Abstract: the ring
+    frees the draft layer's otherwise dead KV pool, room for one more
+    concurrent 1M request).  One fixed KV budget becomes one pool of pages;
+    requests of the 1M workload are admitted through the page allocator
+    (wmtp_pool_alloc, all of a request's pages at once) until it refuses:
+    a native request takes every paged layer's pages (10 target + 1 draft), a
+    windowed one the target layers' pages plus pages worth its ring (the ring
+    itself is a separate tensor of that size).  Each arm's admitted batch is
+    then decoded with page tables taken from the allocator."""
+    import torch
+
+    import synth
+    import speculative_decode_draft_b200 as w
+    base = synth.workload("1m")
+    ctx = int(args.ctx) if args.ctx else base.context[0]
+    Hq, Hkv, D, P, S = base.num_heads_q, base.num_heads_kv, base.head_dim, base.page_size, base.sinks
+    L = args.layers if args.layers is not None else base.verify_layers
+    gamma, W = args.gamma, args.window
+    budget = int(args.kv_budget_gb * 1e9)
+    page_bytes = 2 * Hkv * P * D * 2                      # K and V of one page, bf16
+    num_pages = budget // page_bytes
+    growth = (args.steps + args.warmup) * (gamma + 1)     # tokens the timed and warm-up steps can add
+    p = w.params(Hq, Hkv, D, page_size=P, sinks=S, window=W, gamma_max=gamma)
+    plan = {arm: w.plan_admission(p, ctx + growth, L, 1, arm == "windowed", budget)
+            for arm in ("native", "windowed")}
+    pages_layer = plan["native"]["pages_per_layer"]
+    ring_bytes = plan["windowed"]["draft_bytes"]
+    ring_pages = -(-ring_bytes // page_bytes)
+    # the pool: every page filled with seeded bf16 values once
+    k_pool = torch.empty(num_pages, Hkv, P, D, dtype=torch.bfloat16, device=dev)
+    v_pool = torch.empty_like(k_pool)
+    g = torch.Generator(device=dev)
+    g.manual_seed(base.seed + 1000 * rank + 77)
+    step = max(1, (1 << 30) // (Hkv * P * D * 2))
+    for t in (k_pool, v_pool):
+        for i in range(0, num_pages, step):
+            t[i:i + step].normal_(generator=g)
+    pool = w.PagePool(num_pages)
+    result = {"kv_budget_bytes": budget, "pool_pages": num_pages, "page_bytes": page_bytes,
+              "context": ctx, "target_layers": L, "draft_layers": 1, "gamma": gamma, "window": W,
+              "pages_per_layer": pages_layer, "ring_pages": ring_pages}
+    for arm in ("native", "windowed"):
+        need = (L + 1) * pages_layer if arm == "native" else L * pages_layer + ring_pages
+        admitted = []
+        while True:
+            try:
+                admitted.append(pool.alloc(need))
+            except w.WmtpError:
+                break
+        B = len(admitted)
+        result[f"{arm}_requests"] = B
+        result[f"{arm}_planned_requests"] = plan[arm]["max_requests"]
+        result[f"{arm}_pages_used"] = B * need
+        if B == 0:
+            continue
+
+        def kv(wk, cap, admitted=admitted, arm=arm):
+            # every position a step reads or writes lies in the request's pages
+            assert -(-(int(wk.n_at[-1].max()) + gamma + 1) // P) <= pages_layer
+            lens = torch.tensor(wk.n0s, dtype=torch.int32, device=dev)
+
+            def table(l):
+                rows = [req[l * pages_layer:(l + 1) * pages_layer] for req in admitted]
+                return torch.tensor(rows, dtype=torch.int32, device=dev)
+            caches = [w.PagedCache(k_pool, v_pool, table(l), lens.clone()) for l in range(L)]
+            draft = w.PagedCache(k_pool, v_pool, table(L), lens.clone()) if arm == "native" else None
+            return caches, draft
+        a = argparse.Namespace(**vars(args))
+        a.config, a.ctx = "1m", ctx
+        wk = Workload(a, rank, dev, kv=kv, batch=B)
+        r = time_single_arm(a, wk, arm, world)
+        torch.cuda.synchronize()
+        result[f"{arm}_step_us"] = r["us_per_step"]
+        result[f"{arm}_verify_us_per_layer"] = r["per_call_us"].get("verify")
+        result[f"{arm}_draft_us"] = r["per_call_us"].get("draft")
+        acc = wk.accept[args.warmup:].sum() / args.steps  # accepted tokens per step, whole batch
+        result[f"{arm}_accepted_tokens_per_step"] = float(acc)
+        result[f"{arm}_tokens_per_s"] = float(acc) / (r["us_per_step"] * 1e-6)
+        result[f"{arm}_device_status"] = int(wk.status.item())
+        del wk
+        for req in admitted:
+            pool.release(req)
+        torch.cuda.empty_cache()
+    if rank == 0:
+        line = {"admission": True, "metric": METRIC, "unit": "us/step", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "dtype": "bf16", "data": "synthetic", **result}
+        if result.get("native_tokens_per_s") and result.get("windowed_tokens_per_s"):
+            line["windowed_over_native_throughput"] = result["windowed_tokens_per_s"] / result["native_tokens_per_s"]
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
@@ -656,6 +900,8 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     if args.sweep:
         return run_sweep(args, rank, world, dev)
+    if args.admission:
+        return run_admission(args, rank, world, dev)
     free_bytes, _ = torch.cuda.mem_get_info()  # before the workload's own buffers
     wk = Workload(args, rank, dev)
     stream = torch.cuda.current_stream()
@@ -691,35 +937,38 @@ def main():
     us_nat = ms_nat * 1000.0 / args.steps
 
     # ---------------- end to end: host buffers, copies inside the timed region
+    # Every step's inputs (queries, new K/V, lengths, positions, rollback
+    # targets, bonus counts) start in pinned host memory and are copied in;
+    # every attention output of the step is copied back out.
     e2e = None
     if not args.no_e2e:
         pin = dict(pin_memory=True)
-        h_qd = torch.empty(wk.q_draft[0].shape, dtype=torch.bfloat16, **pin).copy_(wk.q_draft[0])
-        h_qv = torch.empty(wk.q_ver[0].shape, dtype=torch.bfloat16, **pin).copy_(wk.q_ver[0])
-        h_od = torch.empty((wk.gamma,) + tuple(wk.o_draft.shape), dtype=torch.float32, **pin)
-        h_ov = torch.empty((wk.L,) + tuple(wk.o_ver.shape), dtype=torch.float32, **pin)
-        d_qd = torch.empty_like(wk.q_draft[0])
-        d_qv = torch.empty_like(wk.q_ver[0])
-        inputs = {"q_draft": d_qd, "q_ver": d_qv, "out_draft": h_od, "out_ver": h_ov}
+        steps = range(args.warmup, args.warmup + args.steps)
+        host_in = {s: {k: torch.empty(v.shape, dtype=v.dtype, **pin).copy_(v) for k, v in wk.step_inputs(s).items()}
+                   for s in steps}
+        dev_in = {k: torch.empty_like(v) for k, v in wk.step_inputs(args.warmup).items()}
+        outs = {"draft": torch.empty((wk.gamma,) + tuple(wk.o_draft.shape), dtype=torch.float32, **pin),
+                "verify": torch.empty((wk.L,) + tuple(wk.o_ver.shape), dtype=torch.float32, **pin)}
+        h2d = sum(v.numel() * v.element_size() for v in dev_in.values())
+        d2h = sum(v.numel() * v.element_size() for v in outs.values())
         wk.restore_ring(ring_after_warmup)
         barrier(world)
         torch.cuda.synchronize()
-        t0 = time.perf_counter()
         st = torch.cuda.Event(enable_timing=True)
         en = torch.cuda.Event(enable_timing=True)
         st.record()
-        for s in range(args.warmup, args.warmup + args.steps):
-            d_qd.copy_(h_qd, non_blocking=True)
-            d_qv.copy_(h_qv, non_blocking=True)
-            wk.step(s, "windowed", inputs=inputs)
+        for s in steps:
+            for k, v in dev_in.items():
+                v.copy_(host_in[s][k], non_blocking=True)
+            wk.step(s, "windowed", inputs=dev_in, outputs=outs)
         en.record()
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(st.elapsed_time(en), world)
-        h2d = h_qd.numel() * 2 + h_qv.numel() * 2
-        d2h = h_od.numel() * 4 + h_ov.numel() * 4
         e2e = {"value": whole_job_us_per_step(ms_e2e, args.steps, world), "unit": "us/step",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "arm": "windowed"}
-        del t0
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "arm": "windowed",
+               "path": "public Python API (eager launches), inputs copied from pinned host memory and outputs "
+                       "copied back each step"}
+        del host_in, dev_in, outs
 
     torch.cuda.synchronize()
     status = int(wk.status.item())
@@ -742,6 +991,23 @@ def main():
         torch.cuda.synchronize()
         win_paged_us = b0.elapsed_time(b1) * 1000.0 / 10
         del g
+
+    # the windowed draft at 32K, 128K and 1M tokens of context (one sequence,
+    # the ring in the state it has at that length): its time must not grow
+    # with the context
+    flat = None
+    if not args.sweep:
+        from speculative_decode_draft_b200.timing import fill_ring_to, graph_call_us
+        flat = {}
+        q1 = wk.q_draft[args.warmup][0][:1].contiguous()
+        o1, l1 = wk.o_draft[:1], wk.l_draft[:1]
+        for c in (32768, 131072, 1048576):
+            ring = w.Ring.allocate(wk.p, 1, dev)
+            fill_ring_to(wk.p, ring, c, seed=c, device=dev)
+            flat[str(c)] = graph_call_us(lambda: w.draft_attn_windowed(
+                wk.p, q1, ring, out=o1, lse=l1, workspace=wk.workspace, status=wk.status))
+            del ring
+        torch.cuda.empty_cache()
 
     # a read-only streaming reference (torch's sum over 4 GiB; context for the
     # GB/s figures, not a peak the roofline divides by)
@@ -771,14 +1037,13 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = oracle_step_model(args, 524288, repeats=2)
+        units = OracleUnits(args)
+        r = units.step_model()
         cpu = {"value": r["windowed_us"], "unit": "us/step", "cores": cores_used(), "kind": "oracle",
-               "sample": (f"fp64 numpy oracle: one native draft, one windowed draft and one verify layer at "
-                          f"{r['sample_ctx']} tokens (batch 1, 16/2 heads, D=256; draft and verify timed "
-                          f"twice, the faster kept), scaled linearly in context to "
-                          f"{'/'.join(str(c) for c in wk.n0s)} tokens; "
-                          f"{r['work_s']:.1f} s of CPU work"),
-               "native_value": r["native_us"]}
+               "sample": units.sample_desc() + f"; {r['work_s']:.1f} s of timed CPU work",
+               "native_value": r["native_us"], "verify_s_per_layer": r["verify_s"],
+               "draft_native_s": r["draft_native_s"], "draft_windowed_s": r["draft_windowed_s"]}
+        del units
 
     if rank != 0:
         return 0
@@ -810,6 +1075,9 @@ def main():
             "draft_native_us": k_nat["draft"],
             "draft_windowed_us": k_win["draft"],
             "draft_windowed_paged_us": win_paged_us,
+            "draft_windowed_us_by_context": flat,
+            "draft_windowed_spread_by_context": ((max(flat.values()) - min(flat.values())) / statistics.median(
+                flat.values())) if flat else None,
             "verify_us_per_layer": k_win["verify"],
             "verify_us_per_layer_native_arm": k_nat["verify"],
             "draft_native_gbs": nat_gbs,
@@ -820,7 +1088,8 @@ def main():
             "admission": admission,
         },
         "roofline": {"bound": "hbm", "achieved": ver_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": ver_gbs / hbm_peak, "traffic": verify_traffic(workload_desc(args)),
+                     "frac": ver_gbs / hbm_peak,
+                     "traffic": verify_traffic(sum(n + wk.gamma + 1 for n in wk.n0s)),
                      "kernel": "verify_tc_kernel: algorithmic bytes of one verify call / CUDA-event time of the "
                                "call (verify_tc_kernel + its split-KV combine)",
                      "algorithmic_bytes": ver_bytes, "peak_source": peak_src},

@@ -33,9 +33,10 @@
  *   bounded and reports WMTP_DEV_TIMEOUT if it gives up.
  * - bf16 means IEEE bfloat16 (raw 16-bit storage); fp32 accumulation.
  * - Supported shapes: head_dim in {64, 256}; num_heads_q / num_heads_kv = G
- *   with rows = num_q * G in 1..64 (rows are padded to a multiple of 8);
- *   page_size in {16, 32, 64, 128, 256}; gamma_max <= 16.  Anything else
- *   returns WMTP_ERR_UNSUPPORTED.
+ *   with rows = num_q * G in 1..64, or in 1..128 for a verify of head_dim
+ *   256 with num_q >= 2 (gamma = 8 with G = 8 is 72 rows); page_size in
+ *   {16, 32, 64, 128, 256}; gamma_max <= 16; batch and num_heads_kv at most
+ *   65535 (CUDA grid limits).  Anything else returns WMTP_ERR_UNSUPPORTED.
  *
  * Layouts
  * -------
@@ -303,8 +304,14 @@ wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmt
  * library holds that array until the process exits.  The call allocates
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
  *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current).  Make that first call before any
- *     stream capture.
+ *     per device, with that device current; a failed lookup is retried by the
+ *     next call).  Make that first call before any stream capture.
+ *   - The array's device memory is claimed when the library's GPU code is
+ *     loaded on a device.  With CUDA's default lazy module loading that is the
+ *     first call of this library on that device, whichever entry point it is.
+ *     A caller that must have all device memory claimed before a given point
+ *     makes one call per device before it (or sets CUDA_MODULE_LOADING=EAGER,
+ *     which loads the code when the CUDA context is created).
  *   - A call whose scratch would exceed WMTP_NOALLOC_SCRATCH_BYTES returns
  *     WMTP_ERR_WORKSPACE and launches nothing (the size is the one that
  *     wmtp_draft_attn_full reports in *workspace_bytes).

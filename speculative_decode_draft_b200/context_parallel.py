@@ -29,15 +29,24 @@ def slice_query_positions(n_total: torch.Tensor, num_q: int, slice_start: torch.
 
 
 def gather_partials(o_local: torch.Tensor, lse_local: torch.Tensor, group=None):
-    """All-gather every rank's (out, lse) and lay them out as combine
-    partials: part_o ``[rows, world, D]``, part_lse ``[rows, world]``."""
+    """All-gather every rank's (out, lse) in one collective and lay them out as
+    combine partials: part_o ``[rows, world, D]``, part_lse ``[rows, world]``.
+
+    Each rank contributes one ``rows x (D + 1)`` buffer (its output rows with
+    the log-sum-exp appended, in the outputs' dtype: fp32 from the library).
+    A gloo group gathers through host memory."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    go = [torch.empty_like(o_local) for _ in range(world)]
-    gl = [torch.empty_like(lse_local) for _ in range(world)]
-    dist.all_gather(go, o_local.contiguous(), group=group)
-    dist.all_gather(gl, lse_local.contiguous(), group=group)
-    return torch.stack(go, dim=1).contiguous(), torch.stack(gl, dim=1).contiguous()
+    rows, D = o_local.shape
+    packed = torch.cat([o_local, lse_local.to(o_local.dtype).reshape(rows, 1)], dim=1).contiguous()
+    staged = packed.cpu() if (packed.is_cuda and dist.get_backend(group) == "gloo") else packed
+    gathered = torch.empty((world,) + tuple(staged.shape), dtype=staged.dtype, device=staged.device)
+    if staged.is_cuda:
+        dist.all_gather_into_tensor(gathered, staged, group=group)
+    else:
+        dist.all_gather(list(gathered.unbind(0)), staged, group=group)
+    g = gathered.to(o_local.device).permute(1, 0, 2)  # [rows, world, D + 1]
+    return g[:, :, :D].contiguous(), g[:, :, D].contiguous()
 
 
 def verify_attn_context_parallel(p: L.Params, q: torch.Tensor, local_cache: PagedCache,

@@ -72,12 +72,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return pol;
 }
 
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
@@ -202,28 +196,6 @@ __device__ __forceinline__ void commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
 }
-// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16/f16 in, fp32 accumulate).
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// 8 consecutive 32-bit columns of this thread's TMEM lane (32x32b shape: thread
-// i of the warp reads lane base + i), waited for in the same statement so the
-// registers are valid when the statement ends.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
-      : "r"(taddr)
-      : "memory");
-}
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16 (A read from tensor memory).
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -296,29 +268,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v) {
       : "memory");
 }
 
-// NC (a multiple of 8) consecutive columns, in as few loads as possible.
-template <int NC>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NC]) {
-  static_assert(NC % 8 == 0, "columns in multiples of 8");
-#pragma unroll
-  for (int c = 0; c + 32 <= NC; c += 32) tmem_ld32(taddr + c, v + c);
-#pragma unroll
-  for (int c = NC / 32 * 32; c < NC; c += 8) {
-    uint32_t w[8];
-    tmem_ld8(taddr + c, w);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[c + j] = w[j];
-  }
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-      : "memory");
-}
-
 // Shared-memory matrix descriptor (tcgen05 version 1): start address, leading
 // and stride byte offsets (all in 16-byte units), 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -351,14 +300,6 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
-
-// Order-preserving map of a float to a signed int (and back), so a warp can
-// take a float maximum with redux.sync.max.s32.
-__device__ __forceinline__ int float_key(float x) {
-  const int b = __float_as_int(x);
-  return b >= 0 ? b : (b ^ 0x7fffffff);
-}
-__device__ __forceinline__ float key_float(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff)); }
 
 }  // namespace tc
 }  // namespace wmtp

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "ptx.cuh"
 #include "wmtp.h"
@@ -40,7 +41,15 @@ extern "C" wmtp_status wmtp_selftest_wait(int32_t arrive, int32_t* status_word, 
   if (reinterpret_cast<uintptr_t>(cycles_out) % alignof(int64_t) != 0 ||
       reinterpret_cast<uintptr_t>(status_word) % alignof(int32_t) != 0)
     return WMTP_ERR_INVALID_ARG;
-  wmtp::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
-      arrive, status_word, reinterpret_cast<long long*>(cycles_out));
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  // the launch's own return value decides, so an unrelated earlier error left
+  // on this thread cannot be mistaken for a failure of this launch
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(32);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  long long* cyc = reinterpret_cast<long long*>(cycles_out);
+  return cudaLaunchKernelEx(&cfg, wmtp::selftest_wait_kernel, arrive, status_word, cyc) == cudaSuccess
+             ? WMTP_OK
+             : WMTP_ERR_CUDA;
 }

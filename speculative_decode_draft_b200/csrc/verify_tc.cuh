@@ -3,20 +3,23 @@
 // The target verifies gamma+1 draft tokens with causal attention over its
 // full paged KV ("Windowed-MTP ..." arxivlens view, Abstract: verification
 // stays full-context).  All rows = (gamma+1) x G query heads of one KV head
-// share each K/V byte; with G = 8 that is 16..64 rows against every token.
+// share each K/V byte; with G = 8 that is 16..72 rows against every token
+// for gamma = 1..8.
 //
 // Per CTA = (split, KV head, sequence), head_dim 256, 64-token tiles, with
-// the rows as the MMA M dimension (padded to 64) and everything but K and V
+// the rows as the MMA M dimension (padded to M = 64, or to M = 128 for blocks
+// of 65..128 rows such as gamma = 8 with G = 8) and everything but K and V
 // kept in tensor memory (512 columns; the M=64 layout uses lanes 0..15 of
-// each of the four lane quadrants):
+// each of the four lane quadrants, M=128 all 32):
 //   columns   0..127  Q            bf16 pairs, the A operand of S = Q K^T
 //   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax
 //                                  columns 0..31 of the buffer hold P as fp16
 //                                  pairs, the A operand of P V
 //   columns 256..511  O            fp32 output accumulator, 256 head dims
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
-// 16 (r % 4) + r / 4), so the rows spread over the four lane quadrants and
-// each softmax warp owns a quarter of them.
+// 16 (r % 4) + r / 4 for M=64, 32 (r % 4) + r / 4 for M=128), so the rows
+// spread over the four lane quadrants and each softmax warp owns a quarter of
+// them.
 //
 // Roles:
 //   warp 0     streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
@@ -24,10 +27,10 @@
 //              one lane per ring; a K tile is released as soon as its
 //              S = Q K^T has completed, a V tile only after its O += P V, so K
 //              loads run ahead of the softmax;
-//   warp 1     allocates the tensor memory; one lane issues S = Q K^T (M=64,
+//   warp 1     allocates the tensor memory; one lane issues S = Q K^T (M rows,
 //              N=64, K from shared memory, K-major);
-//   warp 10    one lane issues O += P V (M=64, N=256, V read MN-major straight
-//              from the TMA tile).  A lane issues a small tcgen05.mma only
+//   warp 10    one lane issues O += P V (M rows, N=256, V read MN-major
+//              straight from the TMA tile).  A lane issues a small tcgen05.mma only
 //              every ~66 cycles, so the two streams issue from two lanes;
 //   warps 2-5  stage Q into TMEM, then run the softmax, one thread per row:
 //              the row's scores come out of TMEM, the maximum and sum are
@@ -37,14 +40,20 @@
 // The value product is therefore fp16 x fp16 -> fp32: P carries a relative
 // rounding of at most 2^-11 (bf16 would give 2^-8 and miss a 1e-3 relative-L2
 // bound), and V is exact for every |v| < 2^16 (below 2^-17 the absolute error
-// stays under 2^-25); a larger |v| saturates and raises WMTP_DEV_V_RANGE.  One
+// stays under 2^-25); a larger |v| saturates and raises WMTP_DEV_V_RANGE.
+// P is stored as 2^(s - m_ref + 7): the largest weight is then 2^15 (inside
+// fp16's 65504) and weights stay normal fp16 numbers down to 2^-21 of the
+// reference maximum.  Without the offset, a weight below 2^-14 would fall
+// into fp16's subnormal range, where the rounding is absolute (2^-25); a
+// large sea of nearly equal small weights next to one dominant key (an
+// attention sink) would then be rounded the same way and bias the output.  One
 // fp16 MMA per 16 tokens (an N=256 MMA keeps the tensor pipe ~134 cycles)
 // instead of a bf16 hi + lo pair is what keeps PV well under the HBM time of
 // a tile.
 // The reference maximum of a row is raised only when the tile maximum
-// exceeds it by more than 2^8 (weights then stay below 256, well inside
-// fp16), and only then is that row of O rescaled in TMEM, after the previous
-// PV completed.
+// exceeds it by more than 2^8 (with the 2^7 offset, weights then stay at or
+// below 2^15), and only then is that row of O rescaled in TMEM, after the
+// previous PV completed.
 //
 // Every mbarrier wait is bounded; a wait that gives up raises
 // WMTP_DEV_TIMEOUT and stops the pipeline; the producers still wait (bounded)
@@ -69,6 +78,7 @@ constexpr uint32_t kColQ = 0;
 constexpr uint32_t kColS = 128;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;   // lazy rescale threshold (log2 units)
+constexpr float kPShiftLog2 = 7.f;    // P = 2^(s - m_ref + 7) <= 2^15 in fp16
 
 template <int KS, int VS>
 struct TcPlan {
@@ -102,12 +112,15 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
   }
 }
 
-template <int KS, int VS>
+// M: MMA rows (64 or 128); the block's rows must not exceed it.
+template <int KS, int VS, int M>
 __global__ void __launch_bounds__(kTcThreads, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const DecodeArgs a) {
   using Plan = TcPlan<KS, VS>;
   constexpr int D = 256;
+  static_assert(M == 64 || M == 128, "MMA rows: 64 or 128");
+  constexpr int kLanesPerQuadrant = M / 4;  // TMEM lanes of each quadrant that hold rows
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -193,7 +206,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // softmax-thread identity: TMEM lane m = 32 q + lane holds row 4 lane + q
   const int q = warp & 3;
   const int row = 4 * lane + q;
-  const bool row_active = warp >= 2 && warp < 6 && lane < 16 && row < a.rows;
+  const bool row_active = warp >= 2 && warp < 6 && lane < kLanesPerQuadrant && row < a.rows;
   const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
 
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -308,7 +321,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // streams run from two lanes and overlap in the tensor pipe.
   if (warp == kPvWarp) {
     if (lane == 0 && my_tiles > 0) {
-      constexpr uint32_t kIdescPV = tc::idesc_f16_f32(64, 256, 0, 1);    // A (P, TMEM), B (V) MN-major, fp16
+      constexpr uint32_t kIdescPV = tc::idesc_f16_f32(M, 256, 0, 1);     // A (P, TMEM), B (V) MN-major, fp16
       const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffV, Plan::kChunkBytes, 1024);
       bool ok = true;
       for (int k = 0; ok && k < my_tiles; ++k) {
@@ -341,9 +354,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // =================================================================== QK issuer
   if (warp == 1) {
     if (lane == 0 && my_tiles > 0) {
-      // M = 64: the rows never exceed 64, and an M=64 MMA costs the same
-      // issue time as M=128 for half the tensor work (and power)
-      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(64, 64, 0, 0);    // A (Q, TMEM), B (K) K-major
+      // M = 64 whenever the rows fit: an M=64 MMA costs the same issue time
+      // as M=128 for half the tensor work (and power)
+      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(M, 64, 0, 0);     // A (Q, TMEM), B (K) K-major
       // descriptor start addresses are in 16-byte units in the low bits, so
       // moving an operand by n bytes adds n >> 4 to the descriptor
       const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
@@ -464,7 +477,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         moved = m_ref != -INFINITY;
         m_ref = mx;
       }
-      const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const float base = (m_ref == -INFINITY) ? 0.f : m_ref - kPShiftLog2;
       if (__any_sync(0xffffffffu, moved)) {
         // PV(k-1) must have finished before O is rewritten.  S(k) arriving
         // implies PV(k-2) completed (issued before QK(k)), so the pending
@@ -484,7 +497,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc::tmem_st32(tmem_base + lane_addr + kColO + 32 * c, o);
         }
       }
-      // P = 2^(x - base) as fp16 pairs, back into the S columns
+      // P = 2^(x - m_ref + 7) as fp16 pairs, back into the S columns
       float sum = 0.f;
       uint32_t ph[32];
 #pragma unroll
@@ -537,9 +550,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     if (row_active) {
-      // m_ref is in log2 units of the scaled score
+      // m_ref is in log2 units of the scaled score; l_run carries the 2^7
+      // offset of P
       a.part_lse[grow * a.nsplit + split] =
-          (l_run > 0.f && !failed) ? m_ref * 0.69314718055994531f + logf(l_run) : -INFINITY;
+          (l_run > 0.f && !failed) ? (m_ref - kPShiftLog2) * 0.69314718055994531f + logf(l_run) : -INFINITY;
     }
     tc::fence_before_sync();
   }

@@ -6,10 +6,12 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "combine.cuh"
 #include "decode_attn.cuh"
@@ -21,11 +23,13 @@ namespace wmtp {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxRows = 64;
+constexpr int kMaxRows = 64;             // rows per KV head of the mma.sync kernel
+constexpr int kMaxRowsTc = 128;          // rows per KV head of the tcgen05 verify
 constexpr int kMaxGammaMax = 16;
 constexpr int kMaxVerifyWaves = 8;      // CTAs per SM in turn for the tcgen05 verify of a batch
 constexpr int kMinTilesPerSplit = 16;   // extra waves only while full-capacity splits keep this many tiles
 constexpr size_t kWsAlign = 256;
+constexpr int kMaxGridYZ = 65535;       // gridDim.y / gridDim.z limit
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -49,6 +53,47 @@ wmtp_status current_device(int* dev, DeviceInfo* info) {
   if (g_dev[d].sms <= 0) return WMTP_ERR_CUDA;
   *info = g_dev[d];
   return WMTP_OK;
+}
+
+// ---------------------------------------------------------------- launches
+// Dynamic shared-memory opt-in of one kernel, set once per device.  Only a
+// success is remembered: a failed attempt (its error cleared from this
+// library's runtime state) is retried by the next call.  Concurrent first
+// calls from several host threads serialise on the mutex.
+struct SmemAttrOnce {
+  std::atomic<bool> done[kMaxDevices];
+  std::mutex mu;
+};
+
+template <typename Kern>
+wmtp_status ensure_smem_attr(SmemAttrOnce& once, Kern kern, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
+  if (once.done[dev].load(std::memory_order_acquire)) return WMTP_OK;
+  std::lock_guard<std::mutex> lock(once.mu);
+  if (once.done[dev].load(std::memory_order_relaxed)) return WMTP_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return WMTP_ERR_CUDA;
+  }
+  once.done[dev].store(true, std::memory_order_release);
+  return WMTP_OK;
+}
+
+// A launch without attributes whose success is read from the launch call
+// itself, never from cudaGetLastError (which would also report an unrelated
+// earlier error left on this thread, after the kernel had been queued).
+template <typename... Exp, typename... Act>
+wmtp_status launch_plain(void (*kern)(Exp...), dim3 grid, dim3 block, cudaStream_t st, Act&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...) == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -95,10 +140,13 @@ wmtp_status check_params(const wmtp_params* p, int num_q) {
   if (p == nullptr) return WMTP_ERR_INVALID_ARG;
   if (p->num_heads_q <= 0 || p->num_heads_kv <= 0 || num_q <= 0) return WMTP_ERR_INVALID_ARG;
   if (p->num_heads_q % p->num_heads_kv != 0) return WMTP_ERR_INVALID_ARG;
+  if (p->num_heads_kv > kMaxGridYZ) return WMTP_ERR_UNSUPPORTED;
   if (!(p->sm_scale >= 0.f) || !std::isfinite(p->sm_scale)) return WMTP_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 256) return WMTP_ERR_UNSUPPORTED;
-  const int G = p->num_heads_q / p->num_heads_kv;
-  if (static_cast<long long>(G) * num_q > kMaxRows) return WMTP_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(p->num_heads_q / p->num_heads_kv) * num_q;
+  // up to 64 rows on the mma.sync kernel; the tcgen05 verify (head_dim 256,
+  // two or more queries) takes up to 128
+  if (rows > (p->head_dim == 256 && num_q >= 2 ? kMaxRowsTc : kMaxRows)) return WMTP_ERR_UNSUPPORTED;
   return WMTP_OK;
 }
 
@@ -139,10 +187,10 @@ int ctas_per_sm_rt(int D, int NT) {
 // every sequence, so its total work follows the sum of the lengths whatever
 // they are (used by the tcgen05 verify, which is bound per SM by its MMA issue
 // chain; the bandwidth-bound kernels rebalance through the memory system).
-LaunchPlan make_plan(int sms, int B, int Hkv, long long rows_total, int D, int NT, long long max_tiles,
+LaunchPlan make_plan(int sms, int B, int Hkv, long long rows_total, int D, int ctas_per_sm, long long max_tiles,
                      int waves = 1) {
   LaunchPlan pl;
-  const long long slots = static_cast<long long>(sms) * ctas_per_sm_rt(D, NT) * waves;
+  const long long slots = static_cast<long long>(sms) * ctas_per_sm * waves;
   long long per = slots / (static_cast<long long>(B) * Hkv);
   if (waves > 1 && per > max_tiles / kMinTilesPerSplit) per = max_tiles / kMinTilesPerSplit;
   if (per < 1) per = 1;
@@ -184,14 +232,9 @@ wmtp_status launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const 
   constexpr int alloc = SmemPlan<D, NT, S>::kAlloc;
   static_assert(alloc <= kSmemLimit, "shared-memory plan exceeds the sm_100 per-block limit");
   auto kern = decode_attn_kernel<D, NT, S, RING>;
-  static bool attr_done[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
-  if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc) != cudaSuccess)
-      return WMTP_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  static SmemAttrOnce once;
+  const wmtp_status s = ensure_smem_attr(once, kern, alloc);
+  if (s != WMTP_OK) return s;
   return launch_programmatic(kern, dim3(a.nsplit, a.Hkv, B), kThreads, alloc, st, tk, tv, a);
 }
 
@@ -209,24 +252,27 @@ wmtp_status launch_decode(int D, int NT, const CUtensorMap& tk, const CUtensorMa
   return WMTP_ERR_UNSUPPORTED;
 }
 
-wmtp_status launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
-                             cudaStream_t st) {
+template <int M>
+wmtp_status launch_verify_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
+                               cudaStream_t st) {
   constexpr int alloc = TcPlan<kTcKStages, kTcVStages>::kAlloc;
   static_assert(alloc <= kSmemLimit, "shared-memory plan exceeds the sm_100 per-block limit");
-  auto kern = verify_tc_kernel<kTcKStages, kTcVStages>;
-  static bool attr_done[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
-  if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc) != cudaSuccess)
-      return WMTP_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  auto kern = verify_tc_kernel<kTcKStages, kTcVStages, M>;
+  static SmemAttrOnce once;
+  const wmtp_status s = ensure_smem_attr(once, kern, alloc);
+  if (s != WMTP_OK) return s;
   return launch_programmatic(kern, dim3(a.nsplit, a.Hkv, B), kTcThreads, alloc, st, tk, tv, a);
 }
 
-// Verify blocks of head_dim 256 with 9..64 query rows run on tcgen05.
-bool use_verify_tc(int D, int num_q, int rows) { return D == 256 && num_q >= 2 && rows >= 9 && rows <= 64; }
+// M = 64 MMAs while the rows fit (half the tensor work of M = 128 at the
+// same issue cost), M = 128 for 65..128 rows.
+wmtp_status launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
+                             cudaStream_t st) {
+  return a.rows <= 64 ? launch_verify_tc_t<64>(tk, tv, a, B, st) : launch_verify_tc_t<128>(tk, tv, a, B, st);
+}
+
+// Verify blocks of head_dim 256 with 9..128 query rows run on tcgen05.
+bool use_verify_tc(int D, int num_q, int rows) { return D == 256 && num_q >= 2 && rows >= 9 && rows <= kMaxRowsTc; }
 
 // `after_decode`: launched right behind a decode kernel on the same stream, as
 // its programmatic dependent (the combine waits in-kernel for the partials).
@@ -265,9 +311,12 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
   const int rows = num_q * G;
   const int NT = (rows + 7) / 8;
   const long long rows_total = static_cast<long long>(B) * num_q * p->num_heads_q;
+  if (rows_total > 0x7fffffffLL) return WMTP_ERR_UNSUPPORTED;  // the combine's grid x
   const bool tc = !RING && use_verify_tc(D, num_q, rows);
   const int waves = tc ? (B < kMaxVerifyWaves ? B : kMaxVerifyWaves) : 1;
-  LaunchPlan pl = make_plan(info.sms, B, p->num_heads_kv, rows_total, D, NT, max_tiles < 1 ? 1 : max_tiles, waves);
+  const int per_sm = tc ? 1 : ctas_per_sm_rt(D, NT);  // the tcgen05 verify holds a whole SM
+  LaunchPlan pl = make_plan(info.sms, B, p->num_heads_kv, rows_total, D, per_sm, max_tiles < 1 ? 1 : max_tiles,
+                            waves);
   if (workspace == nullptr) {
     *workspace_bytes = pl.bytes;
     return WMTP_OK;
@@ -303,6 +352,7 @@ wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, 
   if (s != WMTP_OK) return s;
   if (window && (num_q != 1 || p->sinks < 0 || p->window < 1)) return WMTP_ERR_INVALID_ARG;
   if (batch < 0 || kv == nullptr || workspace_bytes == nullptr) return WMTP_ERR_INVALID_ARG;
+  if (batch > kMaxGridYZ) return WMTP_ERR_UNSUPPORTED;
   if (!supported_page(p->page_size)) return WMTP_ERR_UNSUPPORTED;
   if (kv->num_pages <= 0 || kv->max_pages <= 0) return WMTP_ERR_INVALID_ARG;
   const long long max_tokens = static_cast<long long>(kv->max_pages) * p->page_size;
@@ -447,6 +497,7 @@ wmtp_status wmtp_draft_attn_windowed(const wmtp_params* params, const void* q, c
   if (s != WMTP_OK) return s;
   if (workspace_bytes == nullptr) return WMTP_ERR_INVALID_ARG;
   const int B = ring->batch;
+  if (B > kMaxGridYZ) return WMTP_ERR_UNSUPPORTED;
   if (B == 0) {
     if (workspace == nullptr) *workspace_bytes = 0;
     return WMTP_OK;
@@ -486,10 +537,9 @@ wmtp_status wmtp_ring_append(const wmtp_params* params, const wmtp_ring* ring, c
   if (speculative && params->gamma_max == 0 && max_new > 0) return WMTP_ERR_INVALID_ARG;
   if (ring->batch == 0) return WMTP_OK;
   RingArgs a = ring_args(params, ring);
-  ring_append_kernel<<<ring->batch, kRingThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      a, truncate_to, n_new, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), max_new,
-      speculative ? 1 : 0, status_word);
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  return launch_plain(ring_append_kernel, dim3(ring->batch), dim3(kRingThreads), static_cast<cudaStream_t>(stream),
+                      a, truncate_to, n_new, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                      max_new, speculative ? 1 : 0, status_word);
 }
 
 wmtp_status wmtp_ring_reset(const wmtp_params* params, const wmtp_ring* ring, void* stream) {
@@ -497,8 +547,7 @@ wmtp_status wmtp_ring_reset(const wmtp_params* params, const wmtp_ring* ring, vo
   if (s != WMTP_OK) return s;
   if (ring->batch == 0) return WMTP_OK;
   RingArgs a = ring_args(params, ring);
-  ring_reset_kernel<<<256, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  return launch_plain(ring_reset_kernel, dim3(256), dim3(256), static_cast<cudaStream_t>(stream), a);
 }
 
 wmtp_status wmtp_splitkv_combine(int32_t rows, int32_t head_dim, int32_t nsplit, const float* part_o,
@@ -519,17 +568,17 @@ wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmt
   if (params->num_heads_kv <= 0 || !supported_page(params->page_size)) return WMTP_ERR_UNSUPPORTED;
   if (params->head_dim <= 0 || params->head_dim % 8 != 0) return WMTP_ERR_UNSUPPORTED;
   if (batch == 0 || n_new == 0) return WMTP_OK;
+  if (batch > kMaxGridYZ) return WMTP_ERR_UNSUPPORTED;
   if (kv->k_pool == nullptr || kv->v_pool == nullptr || kv->page_table == nullptr || pos0 == nullptr ||
       k_new == nullptr || v_new == nullptr)
     return WMTP_ERR_INVALID_ARG;
   if (!aligned(kv->k_pool, 16) || !aligned(kv->v_pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
     return WMTP_ERR_INVALID_ARG;
-  dim3 grid(n_new, batch);
-  paged_write_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(kv->k_pool), static_cast<uint4*>(kv->v_pool), kv->num_pages, kv->page_table,
-      kv->max_pages, params->page_size, params->num_heads_kv, params->head_dim, pos0, n_new,
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), status_word);
-  return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+  return launch_plain(paged_write_kernel, dim3(n_new, batch), dim3(128), static_cast<cudaStream_t>(stream),
+                      static_cast<uint4*>(kv->k_pool), static_cast<uint4*>(kv->v_pool), kv->num_pages,
+                      kv->page_table, kv->max_pages, params->page_size, params->num_heads_kv, params->head_dim,
+                      pos0, n_new, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                      status_word);
 }
 
 }  // extern "C"
@@ -552,9 +601,25 @@ namespace {
 // Device address of the array on each device.  In host code the array's name
 // is only a host-side stand-in, so the real address is fetched once per
 // device, with that device current, and passed to the kernels.
-void* g_noalloc_ptr[kMaxDevices] = {};
-cudaError_t g_noalloc_err[kMaxDevices] = {};
-std::once_flag g_noalloc_once[kMaxDevices];
+// Only a successful lookup is kept; a failed one (for example inside a stream
+// capture) clears its error from this library's runtime state and is retried
+// by the next call.
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+void* noalloc_scratch(int dev) {
+  void* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (ptr != nullptr) return ptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  ptr = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+  if (ptr != nullptr) return ptr;
+  if (cudaGetSymbolAddress(&ptr, wmtp_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+  return ptr;
+}
 
 }  // namespace
 }  // namespace wmtp
@@ -564,12 +629,8 @@ extern "C" wmtp_status wmtp_draft_attn_full_noalloc(const wmtp_params* params, i
                                                     float* lse_out, int32_t* status_word, void* stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WMTP_ERR_CUDA;
-  std::call_once(g_noalloc_once[dev], [dev]() {
-    void* ptr = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, wmtp_noalloc_scratch);
-    g_noalloc_ptr[dev] = ptr;
-  });
-  if (g_noalloc_err[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return WMTP_ERR_CUDA;
+  void* scratch = noalloc_scratch(dev);
+  if (scratch == nullptr) return WMTP_ERR_CUDA;
   size_t need = 0;
   wmtp_status s = paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, nullptr, &need,
                                   status_word, stream);
@@ -577,6 +638,6 @@ extern "C" wmtp_status wmtp_draft_attn_full_noalloc(const wmtp_params* params, i
   if (need > static_cast<size_t>(WMTP_NOALLOC_SCRATCH_BYTES)) return WMTP_ERR_WORKSPACE;
   if (batch == 0) return WMTP_OK;
   size_t have = WMTP_NOALLOC_SCRATCH_BYTES;
-  return paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, g_noalloc_ptr[dev], &have,
-                         status_word, stream);
+  return paged_attention(params, batch, 1, q, kv, out, out_fp32, lse_out, scratch, &have, status_word,
+                         stream);
 }

@@ -74,7 +74,8 @@ def _full(lib, p, batch=1, num_q=None, kv=True):
     (dict(page_size=8), L.WMTP_ERR_UNSUPPORTED),
     (dict(sm_scale=-1.0), L.WMTP_ERR_INVALID_ARG),
     (dict(sm_scale=float("nan")), L.WMTP_ERR_INVALID_ARG),
-    (dict(num_heads_q=128, num_heads_kv=1), L.WMTP_ERR_UNSUPPORTED),  # 128 rows
+    (dict(num_heads_q=128, num_heads_kv=1), L.WMTP_ERR_UNSUPPORTED),  # a 128-row draft
+    (dict(num_heads_q=140000, num_heads_kv=70000), L.WMTP_ERR_UNSUPPORTED),  # grid y limit
 ])
 def test_paged_attention_rejects_bad_params(lib, kw, code):
     assert _full(lib, _p(**kw)) == code
@@ -85,7 +86,9 @@ def test_paged_attention_rejects_missing_pointers(lib):
     assert _full(lib, _p(), kv=False) == L.WMTP_ERR_INVALID_ARG
     assert _full(lib, _p(), batch=-1) == L.WMTP_ERR_INVALID_ARG
     assert _full(lib, _p(), num_q=0) == L.WMTP_ERR_INVALID_ARG
-    assert _full(lib, _p(), num_q=9) == L.WMTP_ERR_UNSUPPORTED  # 9 * 8 = 72 rows
+    assert _full(lib, _p(), num_q=17) == L.WMTP_ERR_UNSUPPORTED  # 17 * 8 = 136 rows
+    assert _full(lib, _p(head_dim=64), num_q=9) == L.WMTP_ERR_UNSUPPORTED  # 72 rows need head_dim 256
+    assert _full(lib, _p(), batch=65536) == L.WMTP_ERR_UNSUPPORTED  # grid z limit
 
 
 def test_batch_zero_is_a_noop(lib):
@@ -122,6 +125,8 @@ def test_combine_and_paged_write_reject_bad_args(lib):
     assert lib.wmtp_paged_write(byref(_p(page_size=3)), 1, byref(desc), None, 1, None, None, None,
                                 None) == L.WMTP_ERR_UNSUPPORTED
     assert lib.wmtp_paged_write(byref(_p()), 1, byref(desc), None, 0, None, None, None, None) == 0
+    assert lib.wmtp_paged_write(byref(_p()), 65536, byref(desc), None, 1, None, None, None,
+                                None) == L.WMTP_ERR_UNSUPPORTED  # grid y limit
 
 
 def test_python_binding_raises_on_wrong_tensors():
@@ -153,8 +158,8 @@ def test_windowed_paged_and_slice_reject_bad_args(lib):
     assert lib.wmtp_verify_attn_slice(byref(_p()), 1, 4, None, byref(desc), None, None, 1, None,
                                       ctypes.addressof(ws) // 256 * 256 + 256, byref(have), None,
                                       None) == L.WMTP_ERR_INVALID_ARG
-    assert lib.wmtp_verify_attn_slice(byref(_p()), 1, 9, None, byref(desc), None, None, 1, None, None,
-                                      byref(size), None, None) == L.WMTP_ERR_UNSUPPORTED  # 72 rows
+    assert lib.wmtp_verify_attn_slice(byref(_p()), 1, 17, None, byref(desc), None, None, 1, None, None,
+                                      byref(size), None, None) == L.WMTP_ERR_UNSUPPORTED  # 136 rows
 
 
 def test_selftest_wait_rejects_misaligned_pointers(lib):

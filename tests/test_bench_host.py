@@ -44,9 +44,11 @@ def test_workload_strings():
 
 
 def test_traffic_guard_follows_the_kernel_code(tmp_path, monkeypatch):
-    desc = bench.workload_desc(bench.parse([]))
-    assert bench.verify_traffic(desc) == bench.VERIFY_TRAFFIC["bytes"]
-    assert bench.verify_traffic(desc.replace("W=4096", "W=1024")) is None  # another workload
+    # a figure recorded against the current sources, 100 bytes per token
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "sha256", bench.kernel_code_hash())
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "tokens", 1000)
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "bytes", 100000)
+    assert bench.verify_traffic(4000) == pytest.approx(400000)  # scaled by tokens
     # a copy of the sources: a comment edit keeps the figure, a code edit drops it
     for rel in bench.VERIFY_TRAFFIC["sources"]:
         os.makedirs(tmp_path / os.path.dirname(rel), exist_ok=True)
@@ -55,9 +57,11 @@ def test_traffic_guard_follows_the_kernel_code(tmp_path, monkeypatch):
     src = tmp_path / bench.VERIFY_TRAFFIC["sources"][0]
     text = src.read_text()
     src.write_text("// a new comment\n" + text)
-    assert bench.verify_traffic(desc) == bench.VERIFY_TRAFFIC["bytes"]
+    assert bench.verify_traffic(4000) == pytest.approx(400000)
     src.write_text(text.replace("kRescaleLog2 = 8.f", "kRescaleLog2 = 7.f"))
-    assert bench.verify_traffic(desc) is None
+    assert bench.verify_traffic(4000) is None
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "bytes", None)
+    assert bench.verify_traffic(4000) is None
 
 
 def test_whole_job_time_per_step():

@@ -2,10 +2,11 @@
 each verified with wmtp_verify_attn_slice, merged with wmtp_splitkv_combine,
 against the fp64 oracle's verify over the whole context.
 
-The ranks of a real context-parallel run each hold one slice; here every
-slice is a page-aligned range of the same pool, so the slices run one after
-the other on one device and only the all-gather is left out (tested on CPU
-with gloo ranks in test_context_parallel_host.py).
+The first test cuts contexts into page-aligned slices of one pool and runs
+them one after the other on one device.  The last one runs the public entry
+point, verify_attn_context_parallel, as two processes on cuda:0 whose
+partials meet in one gloo all-gather, and compares both ranks' merged
+results with the oracle's verify over the whole context.
 """
 
 import numpy as np
@@ -106,3 +107,88 @@ def test_slice_after_a_query_gives_empty_rows():
     assert np.all(np.isinf(l[0])) and np.all(l[0] < 0)      # query 0: position -1 of the slice, nothing
     assert np.all(np.isfinite(l[1:]))
     assert np.all(f64(o)[0, 0] == 0)
+
+
+# ---------------------------------------------------------------- the public entry point, two ranks
+def _cp_rank(rank, world, port, q):
+    """One rank of a two-rank context-parallel verify on cuda:0: it holds
+    positions [rank * n/2, (rank + 1) * n/2) of one 128K-token sequence in its
+    own cache and calls verify_attn_context_parallel; the ranks' partials meet
+    in one gloo all-gather.  The two processes share the GPU, but no kernel of
+    one waits on the other: the exchange happens on the host."""
+    import os
+    import sys
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    try:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        import synth
+        import speculative_decode_draft_b200 as w
+        from speculative_decode_draft_b200.context_parallel import verify_attn_context_parallel
+        torch.cuda.set_device(0)
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        D, G, Hkv, P, num_q, n = 256, 8, 2, 64, 4, 131076
+        p = w.params(G * Hkv, Hkv, D, page_size=P, gamma_max=num_q - 1)
+        kv = synth.paged_kv(71, 1, Hkv, D, P, [n], n + P, True, True, device="cuda:0")
+        qv = synth.queries(72, (1, num_q, G * Hkv, D), device="cuda:0")
+        cut = 65536  # page-aligned: rank 0 holds [0, 65536), rank 1 the rest (with the queries)
+        lo, hi = (0, cut) if rank == 0 else (cut, n)
+        npg = -(-(hi - lo) // P)
+        local = w.PagedCache(kv.k_pool, kv.v_pool, kv.page_table[:, lo // P:lo // P + npg].contiguous(),
+                             torch.tensor([hi - lo], dtype=torch.int32, device="cuda:0"))
+        status = w.new_status("cuda:0")
+        out, lse = verify_attn_context_parallel(
+            p, qv, local, torch.tensor([lo], dtype=torch.int32, device="cuda:0"),
+            torch.tensor([n], dtype=torch.int32, device="cuda:0"), status=status)
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+        q.put((rank, int(status.item()), out.cpu().double().numpy(), lse.cpu().double().numpy()))
+    except BaseException as e:  # report, never hang the parent
+        q.put((rank, "error", repr(e), None))
+
+
+@pytest.mark.timeout(600)
+def test_verify_attn_context_parallel_two_ranks_match_the_oracle():
+    import multiprocessing as mp
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    ps = [ctx.Process(target=_cp_rank, args=(r, 2, port, q)) for r in range(2)]
+    for proc in ps:
+        proc.start()
+    res = {}
+    try:
+        for _ in ps:
+            rank, *rest = q.get(timeout=480)
+            res[rank] = rest
+    finally:
+        for proc in ps:
+            proc.join(timeout=60)
+            if proc.is_alive():
+                proc.kill()
+    for rank in (0, 1):
+        assert res[rank][0] != "error", res[rank]
+        assert res[rank][0] == 0, f"rank {rank}: device status {res[rank][0]:#x}"
+    # the oracle over the whole context, from the same seeded inputs
+    D, G, Hkv, P, num_q, n = 256, 8, 2, 64, 4, 131076
+    kv = synth.paged_kv(71, 1, Hkv, D, P, [n], n + P, True, True, device=DEV)
+    qv = synth.queries(72, (1, num_q, G * Hkv, D), device=DEV)
+    lengths = np.repeat([len(oracle.causal_positions(n, num_q, i)) for i in range(num_q)], G)
+    from _helpers import dense_kv_f64
+    for kvh in range(Hkv):
+        K, V = dense_kv_f64(kv, 0, n, kvh)
+        rows = slice(kvh * G, (kvh + 1) * G)
+        ref, ref_lse = oracle.attend_prefixes(f64(qv[0, :, rows]).reshape(num_q * G, D), K, V, lengths, 1 / 16)
+        for rank in (0, 1):
+            out, lse = res[rank][1], res[rank][2]
+            assert_close(out[0, :, rows].reshape(num_q * G, D), ref, f"context parallel rank {rank} kvh {kvh}")
+            assert_lse_close(lse[0, :, rows].reshape(-1), ref_lse, f"context parallel rank {rank} kvh {kvh}")

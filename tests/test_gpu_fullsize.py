@@ -63,7 +63,8 @@ def _windowed_ref(q, K, V, length, S, W, G, kvh):
 
 # ---------------------------------------------------------------- 128K / 1M
 @pytest.mark.timeout(1200)
-@pytest.mark.parametrize("name,gamma,window", [("128k", 3, 2048), ("1m", 3, 4096), ("1m", 5, 1024)])
+@pytest.mark.parametrize("name,gamma,window", [("128k", 3, 2048), ("1m", 3, 4096), ("1m", 5, 1024),
+                                               ("1m", 8, 4096)])
 def test_fullsize_sampled(name, gamma, window):
     wl = synth.workload(name)
     n0, Hq, Hkv, D, P, S = wl.context[0], wl.num_heads_q, wl.num_heads_kv, wl.head_dim, wl.page_size, wl.sinks
