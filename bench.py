@@ -735,8 +735,8 @@ def run_sweep(args, rank: int, world: int, dev) -> int:
 
     import torch
     contexts = (2048, 8192, 32768, 131072, 524288, 1048576)
-    points = [(c, g, 2048) for c in contexts for g in (1, 3, 5, 7)]
-    points += [(c, 3, W) for c in contexts for W in (1024, 4096, 8192)]
+    points = [(c, g, 2048) for c in contexts for g in (1, 3, 5, 8)]
+    points += [(c, 3, W) for c in (32768, 1048576) for W in (1024, 4096, 8192)]
     for ctx, gamma, window in points:
         a = copy.copy(args)
         a.config, a.ctx, a.gamma, a.window = "1m", ctx, gamma, window

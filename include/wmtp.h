@@ -78,9 +78,8 @@ typedef enum {
                                    truncate_to outside [committed, len] */
 #define WMTP_DEV_UNDO_FULL 0x8  /* speculative appends beyond gamma_max */
 #define WMTP_DEV_TIMEOUT 0x10   /* a bounded in-kernel wait gave up */
-#define WMTP_DEV_V_RANGE 0x20   /* wmtp_verify_attn met a V value with |v| >= 2^16:
-                                   its value product runs in fp16 (exact below
-                                   2^16) and saturated that value */
+#define WMTP_DEV_V_RANGE 0x20   /* reserved: no call sets it (the verify's value
+                                   product takes V in bf16, at any magnitude) */
 
 typedef struct {
   int32_t num_heads_q;  /* Hq */

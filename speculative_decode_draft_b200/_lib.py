@@ -25,7 +25,7 @@ DEV_LEN_OOB = 0x2
 DEV_RING_STATE = 0x4
 DEV_UNDO_FULL = 0x8
 DEV_TIMEOUT = 0x10
-DEV_V_RANGE = 0x20
+DEV_V_RANGE = 0x20  # reserved, never set
 WAIT_LIMIT_CYCLES = 4000000000  # WMTP_WAIT_LIMIT_CYCLES
 
 EXPORTS = (

@@ -29,10 +29,6 @@ __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-__device__ __forceinline__ void grid_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 template <bool OUT_F32>
 __global__ void __launch_bounds__(kCombineThreads)
     splitkv_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,

@@ -42,6 +42,14 @@
 // Masking is by selection (score := -inf), never by multiplication, and V rows
 // past the valid length are zeroed in shared memory, so stale or non-finite
 // bytes beyond a sequence never reach the output.
+//
+// Accumulation runs: a tensor-core MMA adds its products to the fp32
+// accumulator at the accumulator's precision, so products far smaller than
+// the running sum lose low-order bits.  Over a long split of nearly equal
+// weights and values of one sign that loss is systematic (~n 2^-25 of the
+// result after n tokens).  Every kRunTiles tiles the accumulator is therefore
+// folded into the split's fp32 partial in global memory with exact fp32 adds
+// and restarted, so one accumulation spans at most 8,192 tokens.
 #pragma once
 
 #include <cuda.h>
@@ -59,6 +67,7 @@ constexpr int kThreads = 32 * (kComputeWarps + 1);
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kPPitchBytes = 144;  // one P row: 64 bf16 + 16 bytes of padding
 constexpr int kBarCompute = 1;     // named barrier id of the compute warps
+constexpr int kRunTiles = 128;     // tiles per accumulation run (8,192 tokens)
 
 // Status bits (mirror include/wmtp.h).
 constexpr int kDevPageOob = 0x1;
@@ -66,7 +75,6 @@ constexpr int kDevLenOob = 0x2;
 constexpr int kDevRingState = 0x4;
 constexpr int kDevUndoFull = 0x8;
 constexpr int kDevTimeout = 0x10;
-constexpr int kDevVRange = 0x20;
 
 struct DecodeArgs {
   const __nv_bfloat16* q;  // [B][num_q][Hq][D]
@@ -173,7 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_mbar_init();
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
-
   // ---- the token range of this split (uniform across the CTA)
   int n_tok = 0;
   int seq_len = 0;
@@ -210,6 +217,72 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_begin = min(split * tps, ntiles);
   const int t_end = min(t_begin + tps, ntiles);
   const int my_tiles = t_end - t_begin;
+
+  // ---- producer: tile k of the split goes to stage k % STAGES
+  const int box_rows = RING ? kTileTokens : min(a.page_size, kTileTokens);
+  const int boxes = kTileTokens / box_rows;
+  // the page-table entries of tile k (boxes of them; -1 past the sequence),
+  // read one tile ahead of their use so the round trip overlaps the wait for
+  // a free stage
+  auto pages_of = [&](int k, int (&pg)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tok = tile_of(t_begin + k) * kTileTokens + j * box_rows;
+      pg[j] = (!RING && k < my_tiles && j < boxes && tok < n_tok)
+                  ? a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size]
+                  : -1;
+    }
+  };
+  auto produce = [&](int k, const int (&pg)[4]) {
+    const uint64_t pol = ptx::policy_evict_first();
+    const int stage = k % STAGES;
+    const int oob_z = RING ? 0x7fffffff : a.num_pages * a.Hkv;  // past the tensor: zero fill
+    const int tile = tile_of(t_begin + k);
+    const uint32_t kdst = sbase + Plan::kOffK + stage * Plan::kStageBytes;
+    const uint32_t vdst = kdst + Plan::kTileBytes;
+    const uint32_t fb = bar_full + 8 * stage;
+    int valid = 1;
+    if (RING) {
+      stage_flag[stage] = 1;
+      ptx::mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+      const int z = b * a.Hkv + kvh;
+#pragma unroll
+      for (int c = 0; c < Plan::kChunks; ++c) {
+        ptx::tma_load_3d(kdst + c * Plan::kChunkBytes, &tmap_k, fb, c * 64, tile * kTileTokens, z, pol);
+        ptx::tma_load_3d(vdst + c * Plan::kChunkBytes, &tmap_v, fb, c * 64, tile * kTileTokens, z, pol);
+      }
+    } else {
+      // resolve the pages of this tile first, so the validity flag is
+      // published together with the barrier arrival
+      int zs[4];
+      int ys[4];
+      const int tok0 = tile * kTileTokens;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int tok = tok0 + j * box_rows;
+        zs[j] = oob_z;
+        ys[j] = 0;
+        if (j >= boxes || tok >= n_tok) continue;
+        if (pg[j] < 0 || pg[j] >= a.num_pages) {
+          valid = 0;
+        } else {
+          zs[j] = pg[j] * a.Hkv + kvh;
+          ys[j] = tok % a.page_size;
+        }
+      }
+      if (!valid) set_status(a.status, kDevPageOob);
+      stage_flag[stage] = valid;
+      ptx::mbar_arrive_expect_tx(fb, Plan::kStageBytes);
+      for (int j = 0; j < boxes; ++j) {
+#pragma unroll
+        for (int c = 0; c < Plan::kChunks; ++c) {
+          const uint32_t off = c * Plan::kChunkBytes + j * box_rows * 128;
+          ptx::tma_load_3d(kdst + off, &tmap_k, fb, c * 64, ys[j], zs[j], pol);
+          ptx::tma_load_3d(vdst + off, &tmap_v, fb, c * 64, ys[j], zs[j], pol);
+        }
+      }
+    }
+  };
   __syncthreads();
   // let the dependent combine kernel get scheduled while this grid runs; it
   // waits in-kernel until this grid has finished and its writes are visible
@@ -220,69 +293,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && my_tiles > 0) {
       ptx::prefetch_tmap(&tmap_k);
       ptx::prefetch_tmap(&tmap_v);
-      const uint64_t pol = ptx::policy_evict_first();
-      const int box_rows = RING ? kTileTokens : min(a.page_size, kTileTokens);
-      const int boxes = kTileTokens / box_rows;
-      const int oob_z = RING ? 0x7fffffff : a.num_pages * a.Hkv;  // past the tensor: zero fill
       int issued = 0;
+      int pg_cur[4], pg_nxt[4];
+      pages_of(0, pg_cur);
       for (int k = 0; k < my_tiles; ++k) {
+        // entries four tiles ahead head for L2; the next tile's are read now
+        if (!RING && k + 4 < my_tiles) {
+          const int ahead = tile_of(t_begin + k + 4) * kTileTokens;
+          if (ahead < n_tok)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.page_table + static_cast<size_t>(b) * a.max_pages +
+                                                              ahead / a.page_size));
+        }
+        pages_of(k + 1, pg_nxt);
         const int stage = k % STAGES;
         const uint32_t par = ((k / STAGES) & 1) ^ 1;
         if (!ptx::mbar_wait(bar_empty + 8 * stage, par)) {
           set_status(a.status, kDevTimeout);
           break;
         }
-        const int tile = tile_of(t_begin + k);
-        const uint32_t kdst = sbase + Plan::kOffK + stage * Plan::kStageBytes;
-        const uint32_t vdst = kdst + Plan::kTileBytes;
-        const uint32_t fb = bar_full + 8 * stage;
-        int valid = 1;
-        if (RING) {
-          stage_flag[stage] = 1;
-          ptx::mbar_arrive_expect_tx(fb, Plan::kStageBytes);
-          const int z = b * a.Hkv + kvh;
-#pragma unroll
-          for (int c = 0; c < Plan::kChunks; ++c) {
-            ptx::tma_load_3d(kdst + c * Plan::kChunkBytes, &tmap_k, fb, c * 64, tile * kTileTokens, z, pol);
-            ptx::tma_load_3d(vdst + c * Plan::kChunkBytes, &tmap_v, fb, c * 64, tile * kTileTokens, z, pol);
-          }
-        } else {
-          // resolve the pages of this tile first, so the validity flag is
-          // published together with the barrier arrival
-          int zs[4];
-          int ys[4];
-          const int tok0 = tile * kTileTokens;
-          for (int j = 0; j < boxes; ++j) {
-            const int tok = tok0 + j * box_rows;
-            if (tok >= n_tok) {
-              zs[j] = oob_z;
-              ys[j] = 0;
-              continue;
-            }
-            const int lp = tok / a.page_size;
-            const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + lp];
-            if (pg < 0 || pg >= a.num_pages) {
-              valid = 0;
-              zs[j] = oob_z;
-              ys[j] = 0;
-            } else {
-              zs[j] = pg * a.Hkv + kvh;
-              ys[j] = tok - lp * a.page_size;
-            }
-          }
-          if (!valid) set_status(a.status, kDevPageOob);
-          stage_flag[stage] = valid;
-          ptx::mbar_arrive_expect_tx(fb, Plan::kStageBytes);
-          for (int j = 0; j < boxes; ++j) {
-#pragma unroll
-            for (int c = 0; c < Plan::kChunks; ++c) {
-              const uint32_t off = c * Plan::kChunkBytes + j * box_rows * 128;
-              ptx::tma_load_3d(kdst + off, &tmap_k, fb, c * 64, ys[j], zs[j], pol);
-              ptx::tma_load_3d(vdst + off, &tmap_v, fb, c * 64, ys[j], zs[j], pol);
-            }
-          }
-        }
+        produce(k, pg_cur);
         issued = k + 1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pg_cur[j] = pg_nxt[j];
       }
       // no copy may still be writing shared memory when the CTA exits (after
       // a timeout the consumers stop early): wait, bounded, for the last load
@@ -348,9 +380,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   const int dbase = warp * (D / 4);
+  // the accumulator folded so far (in the split's partial slot, units of
+  // 2^m_g) for each of this thread's rows
+  float m_g[NT][2];
+  bool have_g[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_g[nt][0] = m_g[nt][1] = -INFINITY;
+    have_g[nt][0] = have_g[nt][1] = false;
+  }
+  auto row_dst = [&](int row) -> float* {
+    const size_t grow = (static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G;
+    return a.part_o + (grow * a.nsplit + split) * D;
+  };
   const int first_masked_tok = RING ? -1 : min(n_tok, q_first + 1);  // tokens >= this may be masked
 
   for (int k = 0; k < my_tiles; ++k) {
+    if (k > 0 && (k % kRunTiles) == 0) {
+      // fold the finished run: G = G 2^(m_g - m_run) + O, then restart O
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int row = nt * 8 + 2 * t4 + j;
+          if (row >= a.rows || m_run[nt][j] == -INFINITY) continue;
+          const float gs = have_g[nt][j] ? ptx::ex2(m_g[nt][j] - m_run[nt][j]) : 0.f;
+          float* dst = row_dst(row);
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt) {
+            const int d = dbase + 16 * mt + g;
+            dst[d] = (have_g[nt][j] ? dst[d] * gs : 0.f) + o_acc[mt][nt][j];
+            dst[d + 8] = (have_g[nt][j] ? dst[d + 8] * gs : 0.f) + o_acc[mt][nt][j + 2];
+            o_acc[mt][nt][j] = 0.f;
+            o_acc[mt][nt][j + 2] = 0.f;
+          }
+          m_g[nt][j] = m_run[nt][j];
+          have_g[nt][j] = true;
+        }
+    }
     const int stage = k % STAGES;
     const uint32_t par = (k / STAGES) & 1;
     const bool got = ptx::mbar_wait(bar_full + 8 * stage, par);
@@ -566,15 +633,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int w = 0; w < kComputeWarps; ++w) l += red[w * kRows + row];
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      const int qi = row / a.G;
-      const int hq = kvh * a.G + row % a.G;
-      const size_t grow = (static_cast<size_t>(b) * a.num_q + qi) * a.Hq + hq;
-      float* dst = a.part_o + (grow * a.nsplit + split) * D;
+      const size_t grow = (static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G;
+      float* dst = row_dst(row);
+      const bool hg = have_g[nt][j];
+      const float gs = hg ? ptx::ex2(m_g[nt][j] - m_run[nt][j]) : 0.f;
 #pragma unroll
       for (int mt = 0; mt < kMT; ++mt) {
         const int d = dbase + 16 * mt + g;
-        dst[d] = o_acc[mt][nt][j] * inv;
-        dst[d + 8] = o_acc[mt][nt][j + 2] * inv;
+        dst[d] = ((hg ? dst[d] * gs : 0.f) + o_acc[mt][nt][j]) * inv;
+        dst[d + 8] = ((hg ? dst[d + 8] * gs : 0.f) + o_acc[mt][nt][j + 2]) * inv;
       }
       if (warp == 0 && g == 0) {
         // m_run is in log2 units of the scaled score

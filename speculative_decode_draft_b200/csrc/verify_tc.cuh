@@ -13,8 +13,8 @@
 // each of the four lane quadrants, M=128 all 32):
 //   columns   0..127  Q            bf16 pairs, the A operand of S = Q K^T
 //   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax
-//                                  columns 0..31 of the buffer hold P as fp16
-//                                  pairs, the A operand of P V
+//                                  columns 0..31 of the buffer hold P_hi and
+//                                  32..63 P_lo as bf16 pairs (P = hi + lo)
 //   columns 256..511  O            fp32 output accumulator, 256 head dims
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
 // 16 (r % 4) + r / 4 for M=64, 32 (r % 4) + r / 4 for M=128), so the rows
@@ -22,38 +22,41 @@
 // them.
 //
 // Roles:
-//   warp 0     streams K and V tiles (64 x 256 bf16 each, 128-byte swizzle)
-//              into two shared-memory rings (KS and VS tiles deep) with TMA,
-//              one lane per ring; a K tile is released as soon as its
-//              S = Q K^T has completed, a V tile only after its O += P V, so K
-//              loads run ahead of the softmax;
+//   warps 0, 7 stream K (warp 0) and V (warp 7) tiles (64 x 256 bf16 each,
+//              128-byte swizzle) into two shared-memory rings (KS and VS tiles
+//              deep) with TMA, one lane each; a K tile is released as soon as
+//              its S = Q K^T has completed, a V tile after its O += P V.  The
+//              two producers sit in different warps so that neither one's
+//              barrier wait holds up the other's issue;
 //   warp 1     allocates the tensor memory; one lane issues S = Q K^T (M rows,
 //              N=64, K from shared memory, K-major);
-//   warp 10    one lane issues O += P V (M rows, N=256, V read MN-major
-//              straight from the TMA tile).  A lane issues a small tcgen05.mma only
-//              every ~66 cycles, so the two streams issue from two lanes;
-//   warps 2-5  stage Q into TMEM, then run the softmax, one thread per row:
-//              the row's scores come out of TMEM, the maximum and sum are
-//              taken inside the thread, and P goes back into TMEM in fp16;
-//   warps 6-9  convert each landed V tile in place from bf16 to fp16 (and
-//              zero its rows past the sequence end).
-// The value product is therefore fp16 x fp16 -> fp32: P carries a relative
-// rounding of at most 2^-11 (bf16 would give 2^-8 and miss a 1e-3 relative-L2
-// bound), and V is exact for every |v| < 2^16 (below 2^-17 the absolute error
-// stays under 2^-25); a larger |v| saturates and raises WMTP_DEV_V_RANGE.
-// P is stored as 2^(s - m_ref + 7): the largest weight is then 2^15 (inside
-// fp16's 65504) and weights stay normal fp16 numbers down to 2^-21 of the
-// reference maximum.  Without the offset, a weight below 2^-14 would fall
-// into fp16's subnormal range, where the rounding is absolute (2^-25); a
-// large sea of nearly equal small weights next to one dominant key (an
-// attention sink) would then be rounded the same way and bias the output.  One
-// fp16 MMA per 16 tokens (an N=256 MMA keeps the tensor pipe ~134 cycles)
-// instead of a bf16 hi + lo pair is what keeps PV well under the HBM time of
-// a tile.
+//   warp 6     one lane issues O += P V (M rows, N=256, V read MN-major
+//              straight from the TMA tile, bf16).  A lane issues a small
+//              tcgen05.mma only every ~66 cycles, so the two streams issue
+//              from two lanes;
+//   warps 2-5  stage Q into TMEM, then run the softmax.  Each warp covers the
+//              rows of its lane quadrant with sixteen-lane TMEM accesses: four
+//              threads share a row and take 16 of the tile's 64 scores each,
+//              so every lane of the warp works even when a quadrant holds only
+//              8 rows (gamma = 3, G = 8).  Row maxima meet through two
+//              shuffles; P goes back into TMEM.
+// The value product is bf16 x bf16 -> fp32 on two MMAs per 16 tokens: P is
+// split into P_hi = bf16(p) and P_lo = bf16(p - P_hi), |p - P_hi - P_lo| <=
+// 2^-16 p (a single bf16 P, 2^-8, would miss a 1e-3 relative-L2 bound), and V
+// enters in its own bf16 format, exactly and at any magnitude.
 // The reference maximum of a row is raised only when the tile maximum
-// exceeds it by more than 2^8 (with the 2^7 offset, weights then stay at or
-// below 2^15), and only then is that row of O rescaled in TMEM, after the
-// previous PV completed.
+// exceeds it by more than 2^8 (weights then stay at or below 2^8), and only
+// then is that row of O rescaled in TMEM, after the previous PV completed.
+//
+// Accumulation runs: a tensor-core accumulation adds each product to the
+// fp32 accumulator at the accumulator's precision, so a product far smaller
+// than the running sum loses low-order bits.  Over a long split of nearly
+// equal weights and values of one sign (a flat stretch of attention) that
+// loss is systematic, ~n 2^-25 of the result after n products.  Every
+// kRunTiles tiles the softmax threads therefore fold the accumulator into the
+// split's fp32 partial in global memory (exact fp32 adds) and the next PV
+// starts a fresh accumulation; a run then spans at most 8,192 tokens
+// (kRunTiles, shared with the mma.sync kernel).
 //
 // Every mbarrier wait is bounded; a wait that gives up raises
 // WMTP_DEV_TIMEOUT and stops the pipeline; the producers still wait (bounded)
@@ -70,15 +73,16 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 352;       // producers, QK issuer, 4 softmax warps, 4 V converter warps, PV issuer
-constexpr int kPvWarp = 10;
-constexpr int kBarTmem = 3;           // named barrier: MMA + softmax warps
+constexpr int kTcThreads = 256;       // K producer, QK issuer, 4 softmax warps, PV issuer, V producer
+constexpr int kPvWarp = 6;
+constexpr int kVWarp = 7;
+constexpr int kBarTmem = 3;           // named barrier: QK issuer + softmax warps
+constexpr int kBarSoftmax = 4;        // named barrier: the softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;
 constexpr uint32_t kColS = 128;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;   // lazy rescale threshold (log2 units)
-constexpr float kPShiftLog2 = 7.f;    // P = 2^(s - m_ref + 7) <= 2^15 in fp16
 
 template <int KS, int VS>
 struct TcPlan {
@@ -87,17 +91,15 @@ struct TcPlan {
   static constexpr int kOffK = 0;                         // K ring: KS tiles
   static constexpr int kOffV = KS * kTileBytes;           // V ring: VS tiles
   static constexpr int kOffBar = (KS + VS) * kTileBytes;
-  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], v_ready[VS], s_full[2],
-  // p_full[2], o_done, mma_final, q_ready, pv_done[2]
-  static constexpr int kNumBars = 2 * KS + 3 * VS + 9;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort
-  static constexpr int kBytes = kOffMisc + 8;
+  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
+  // o_done, mma_final, q_ready, pv_done[2]
+  static constexpr int kNumBars = 2 * KS + 2 * VS + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, split page validity
+  static constexpr int kBytes = kOffMisc + 12;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-// Depths of the K and V rings (64-token tiles).  K tiles leave as soon as QK
-// has read them and V tiles only after the softmax and PV, yet 2 + 4 measured
-// slower than 3 + 3 on B200 (398-404 against 393-396 us per 1M layer).
+// Depths of the K and V rings (64-token tiles).
 constexpr int kTcKStages = 3;
 constexpr int kTcVStages = 3;
 
@@ -112,6 +114,13 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
   }
 }
 
+// p0, p1 -> bf16 hi pair and lo pair (p = hi + lo to 2^-16 relative); the
+// first value goes to the low half of each word.
+__device__ __forceinline__ void split_pack(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  hi = ptx::pack_bf16x2(p0, p1);
+  lo = ptx::pack_bf16x2(p0 - ptx::bf16lo_to_f32(hi), p1 - ptx::bf16hi_to_f32(hi));
+}
+
 // M: MMA rows (64 or 128); the block's rows must not exceed it.
 template <int KS, int VS, int M>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -120,7 +129,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using Plan = TcPlan<KS, VS>;
   constexpr int D = 256;
   static_assert(M == 64 || M == 128, "MMA rows: 64 or 128");
-  constexpr int kLanesPerQuadrant = M / 4;  // TMEM lanes of each quadrant that hold rows
+  constexpr int H = M / 64;  // sixteen-lane halves of a quadrant that hold rows
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -131,13 +140,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_k_empty = bar_k_full + 8 * KS;
   const uint32_t bar_v_full = bar_k_empty + 8 * KS;
   const uint32_t bar_v_empty = bar_v_full + 8 * VS;
-  const uint32_t bar_v_ready = bar_v_empty + 8 * VS;
-  const uint32_t bar_s_full = bar_v_ready + 8 * VS;
+  const uint32_t bar_s_full = bar_v_empty + 8 * VS;
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_o_done = bar_p_full + 16;
   const uint32_t bar_final = bar_o_done + 8;
   const uint32_t bar_q_ready = bar_final + 8;
   const uint32_t bar_pv_done = bar_q_ready + 8;  // [2]: PV of the tiles using S/P buffer 0 / 1
+  volatile int* split_bad = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
 
@@ -156,7 +165,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < VS; ++s) {
       ptx::mbar_init(bar_v_full + 8 * s, 1);
       ptx::mbar_init(bar_v_empty + 8 * s, 1);
-      ptx::mbar_init(bar_v_ready + 8 * s, 4);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar_s_full + 8 * i, 1);
@@ -168,6 +176,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ptx::mbar_init(bar_pv_done + 8, 1);
     ptx::mbar_init(bar_q_ready, 4);
     *abort_flag = 0;
+    *split_bad = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -177,7 +186,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // every global-memory access comes after this: with a programmatic launch
   // the set-up above overlaps the previous kernel's tail
   asm volatile("griddepcontrol.wait;" ::: "memory");
-
   // ---- token range of this split
   int n_tok = a.kv_len[b];
   if (n_tok != 0 &&
@@ -190,6 +198,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int t_begin = min(split * tps, ntiles);
   const int t_end = min(t_begin + tps, ntiles);
   const int my_tiles = t_end - t_begin;
+
+  // ---- producers: warp 0 loads K tiles, warp 7 V tiles (lane 0 each), each
+  // into its own ring.  Tile k of a ring goes to stage k % depth.
+  const bool is_k = warp == 0;
+  const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+  const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
+  const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
+  const int nst = is_k ? KS : VS;  // stages of this lane's ring
+  const int box_rows = min(a.page_size, kTileTokens);
+  const int boxes = kTileTokens / box_rows;
+  // the page-table entries of tile k (boxes of them; -1 past the sequence),
+  // read one tile ahead of their use so the round trip overlaps the wait for
+  // a free stage
+  auto pages_of = [&](int k, int (&pg)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tok = (t_begin + k) * kTileTokens + j * box_rows;
+      pg[j] = (k < my_tiles && j < boxes && tok < n_tok)
+                  ? a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size]
+                  : -1;
+    }
+  };
+  auto produce = [&](int k, const int (&pg)[4], uint64_t pol) {
+    const int tok0 = (t_begin + k) * kTileTokens;
+    const int oob_z = a.num_pages * a.Hkv;  // past the tensor: zero fill
+    const uint32_t dst = sbase + (is_k ? Plan::kOffK : Plan::kOffV) + (k % nst) * Plan::kTileBytes;
+    const uint32_t fb = bar_full + 8 * (k % nst);
+    int zs[4], ys[4];
+    int valid = 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tok = tok0 + j * box_rows;
+      zs[j] = oob_z;
+      ys[j] = 0;
+      if (j >= boxes || tok >= n_tok) continue;
+      if (pg[j] < 0 || pg[j] >= a.num_pages) {
+        valid = 0;
+      } else {
+        zs[j] = pg[j] * a.Hkv + kvh;
+        ys[j] = tok % a.page_size;
+      }
+    }
+    if (is_k && !valid) set_status(a.status, kDevPageOob);
+    ptx::mbar_arrive_expect_tx(fb, Plan::kTileBytes);
+    for (int j = 0; j < boxes; ++j) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        ptx::tma_load_3d(dst + c * Plan::kChunkBytes + j * box_rows * 128, tmap, fb, c * 64, ys[j], zs[j], pol);
+    }
+  };
   // start the page-table reads of the first tiles now; the producers' own
   // loads then hit L2
   if (warp == 0 && lane < VS && lane < my_tiles) {
@@ -203,64 +261,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  // softmax-thread identity: TMEM lane m = 32 q + lane holds row 4 lane + q
-  const int q = warp & 3;
-  const int row = 4 * lane + q;
-  const bool row_active = warp >= 2 && warp < 6 && lane < kLanesPerQuadrant && row < a.rows;
-  const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // =================================================================== producers
-  // lane 0 loads K tiles, lane 1 loads V tiles; each has its own ring
-  if (warp == 0) {
-    if (lane < 2 && my_tiles > 0) {
-      const bool is_k = lane == 0;
-      const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+  if (warp == 0 || warp == kVWarp) {
+    if (lane == 0 && my_tiles > 0) {
       ptx::prefetch_tmap(tmap);
       const uint64_t pol = ptx::policy_evict_first();
-      const int box_rows = min(a.page_size, kTileTokens);
-      const int boxes = kTileTokens / box_rows;
-      const int oob_z = a.num_pages * a.Hkv;  // past the tensor: zero fill
-      const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
-      const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
-      const uint32_t ring = sbase + (is_k ? Plan::kOffK : Plan::kOffV);
-      const int nst = is_k ? KS : VS;  // stages of this lane's ring
       int issued = 0;
+      int pg_cur[4], pg_nxt[4];
+      pages_of(0, pg_cur);
       for (int k = 0; k < my_tiles; ++k) {
-        const int stage = k % nst;
-        if (!tc_wait(bar_empty + 8 * stage, ((k / nst) & 1) ^ 1, abort_flag)) {
+        // entries four tiles ahead head for L2; the next tile's are read now
+        const int ahead = (t_begin + k + 4) * kTileTokens;
+        if (k + 4 < my_tiles && ahead < n_tok)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.page_table + static_cast<size_t>(b) * a.max_pages +
+                                                            ahead / a.page_size));
+        pages_of(k + 1, pg_nxt);
+        if (!tc_wait(bar_empty + 8 * (k % nst), ((k / nst) & 1) ^ 1, abort_flag)) {
           if (*abort_flag == 0) set_status(a.status, kDevTimeout);
           *abort_flag = 1;
           break;
         }
-        const int tok0 = (t_begin + k) * kTileTokens;
-        const uint32_t dst = ring + stage * Plan::kTileBytes;
-        const uint32_t fb = bar_full + 8 * stage;
-        int zs[4], ys[4];
-        int valid = 1;
-        for (int j = 0; j < boxes; ++j) {
-          const int tok = tok0 + j * box_rows;
-          zs[j] = oob_z;
-          ys[j] = 0;
-          if (tok >= n_tok) continue;
-          const int lp = tok / a.page_size;
-          const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + lp];
-          if (pg < 0 || pg >= a.num_pages) {
-            valid = 0;
-          } else {
-            zs[j] = pg * a.Hkv + kvh;
-            ys[j] = tok - lp * a.page_size;
-          }
-        }
-        if (is_k && !valid) set_status(a.status, kDevPageOob);
-        ptx::mbar_arrive_expect_tx(fb, Plan::kTileBytes);
-        for (int j = 0; j < boxes; ++j) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            ptx::tma_load_3d(dst + c * Plan::kChunkBytes + j * box_rows * 128, tmap, fb, c * 64, ys[j], zs[j], pol);
-        }
+        produce(k, pg_cur, pol);
         issued = k + 1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pg_cur[j] = pg_nxt[j];
       }
       // no copy may still be writing shared memory when the CTA exits (after
       // an abort the consumers stop early): wait, bounded, for the last load
@@ -271,70 +297,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return;
   }
 
-  // =================================================================== V converters
-  if (warp >= 6 && warp < kPvWarp) {
-    const int cw = warp - 6;  // one 8 KB column chunk (64 head dims) of the V tile per warp
-    uint32_t vexp = 0;        // per-half maximum of the bf16 exponent fields seen
-    for (int k = 0; k < my_tiles; ++k) {
-      const int stage = k % VS;
-      if (!__all_sync(0xffffffffu, tc_wait(bar_v_full + 8 * stage, (k / VS) & 1, abort_flag))) {
-        if (lane == 0) set_status(a.status, kDevTimeout);
-        *abort_flag = 1;
-        break;
-      }
-      const int tok0 = (t_begin + k) * kTileTokens;
-      const int rows_valid = min(kTileTokens, n_tok - tok0);
-      const uint32_t chunk = sbase + Plan::kOffV + stage * Plan::kTileBytes + cw * Plan::kChunkBytes;
-#pragma unroll 4
-      for (int u = lane; u < Plan::kChunkBytes / 16; u += 32) {
-        const uint32_t addr = chunk + 16 * u;
-        uint4 w;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
-                     : "r"(addr));
-        if (u / 8 < rows_valid) {  // 8 sixteen-byte units per 128-byte row
-          vexp = __vmaxu2(vexp, __vmaxu2(w.x & 0x7f807f80u, w.y & 0x7f807f80u));
-          vexp = __vmaxu2(vexp, __vmaxu2(w.z & 0x7f807f80u, w.w & 0x7f807f80u));
-          w.x = ptx::bf16x2_to_f16x2_sat(w.x);
-          w.y = ptx::bf16x2_to_f16x2_sat(w.y);
-          w.z = ptx::bf16x2_to_f16x2_sat(w.z);
-          w.w = ptx::bf16x2_to_f16x2_sat(w.w);
-        } else {  // past the end of the sequence: zero, so 0-weight rows add 0
-          w = make_uint4(0, 0, 0, 0);
-        }
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w.x), "r"(w.y), "r"(w.z),
-                     "r"(w.w)
-                     : "memory");
-      }
-      ptx::fence_proxy_async_smem();  // generic writes before the tensor core reads
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar_v_ready + 8 * stage);
-    }
-    // a bf16 exponent field of 143 or more means |v| >= 2^16
-    if ((vexp & 0xffffu) >= (143u << 7) || (vexp >> 16) >= (143u << 7)) set_status(a.status, kDevVRange);
-    return;
-  }
-
   // =================================================================== PV issuer
   // O += P(k) V(k) for every tile, issued by its own lane: a single lane
   // issues a small tcgen05.mma only every ~66 cycles, so the QK and PV
-  // streams run from two lanes and overlap in the tensor pipe.
+  // streams run from two lanes and overlap in the tensor pipe.  Per 16
+  // tokens two MMAs: P_hi V and P_lo V.  The first MMA of a run starts a
+  // fresh accumulation (the softmax threads have folded the previous run).
   if (warp == kPvWarp) {
     if (lane == 0 && my_tiles > 0) {
-      constexpr uint32_t kIdescPV = tc::idesc_f16_f32(M, 256, 0, 1);     // A (P, TMEM), B (V) MN-major, fp16
+      constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(M, 256, 0, 1);    // A (P, TMEM), B (V) MN-major
       const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffV, Plan::kChunkBytes, 1024);
       bool ok = true;
       for (int k = 0; ok && k < my_tiles; ++k) {
         ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag) &&
-             tc_wait(bar_v_ready + 8 * (k % VS), (k / VS) & 1, abort_flag);
+             tc_wait(bar_v_full + 8 * (k % VS), (k / VS) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
         const uint64_t vd = v_desc0 + (static_cast<uint64_t>((k % VS) * Plan::kTileBytes) >> 4);
         const uint32_t p_tmem = tmem_base + kColS + (k & 1) * 64;
+        const uint32_t fresh = (k % kRunTiles) == 0 ? 0u : 1u;  // 0: overwrite O
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+          // 16 tokens = 8 columns of bf16 pairs; V rows 16 kk .. 16 kk + 15
           const uint64_t bd = vd + (static_cast<uint32_t>(kk * 2048) >> 4);
-          tc::mma_ts(tmem_base + kColO, p_tmem + 8 * kk, bd, kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(tmem_base + kColO, p_tmem + 8 * kk, bd, kIdescPV, kk > 0 ? 1u : fresh);
+          tc::mma_ts(tmem_base + kColO, p_tmem + 32 + 8 * kk, bd, kIdescPV, 1u);
         }
         tc::commit(bar_v_empty + 8 * (k % VS));
         tc::commit(bar_o_done);
@@ -392,17 +379,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ================================================================= softmax
+    const int q = warp & 3;  // this warp's TMEM lane quadrant
+    const uint32_t qlane = static_cast<uint32_t>(32 * q) << 16;
     {
-      // Q row into TMEM columns 0..127 (bf16 pairs), zeros for padding rows;
-      // every load is issued before the first store so the row costs one
-      // global-memory round trip
+      // Q: thread `lane` stages row 4 lane + q into TMEM lane 32 q + lane
+      // (columns 0..127, bf16 pairs), zeros for padding rows; every load is
+      // issued before the first store so the row costs one global round trip
+      const int row = 4 * lane + q;
+      const bool q_active = lane < M / 4 && row < a.rows;
       const __nv_bfloat16* src =
-          row_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
-                     : nullptr;
+          q_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
+                   : nullptr;
       uint4 v[D / 8];
 #pragma unroll
       for (int j = 0; j < D / 8; ++j)
-        v[j] = row_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
+        v[j] = q_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t wq[32];
@@ -413,109 +404,266 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           wq[4 * j + 2] = v[8 * c + j].z;
           wq[4 * j + 3] = v[8 * c + j].w;
         }
-        tc::tmem_st32(tmem_base + lane_addr + kColQ + 32 * c, wq);
+        tc::tmem_st32(tmem_base + qlane + kColQ + 32 * c, wq);
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_q_ready);
     }
-    // query i attends positions <= q_first + i of this cache (q_first is
-    // kv_len - num_q unless the call covers a slice of a longer sequence)
+
+    // Sixteen-lane view: in half h this thread covers TMEM lanes
+    // 16 h + lane / 4 (sub-row j = 0) and 16 h + lane / 4 + 8 (j = 1) of the
+    // quadrant, and columns 8 r + 2 (lane % 4) + {0, 1} of every 8 (r = 0..7).
+    // The four threads lane / 4 * 4 + {0..3} share both rows.
+    const int cq = 2 * (lane & 3);
+    int row_of[H][2];
+    bool act[H][2];    // this thread's row exists
+    bool any_r[H][2];  // some row of this warp's (half, sub-row) group exists (warp-uniform)
+    int lim[H][2];     // causal limit (exclusive)
     const int q_first = a.q_pos0 != nullptr ? a.q_pos0[b] : n_tok - a.num_q;
-    const int lim = row_active ? min(n_tok, q_first + row / a.G + 1) : n_tok;  // causal limit of this row
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int ln = 16 * h + 8 * j + (lane >> 2);  // lane inside the quadrant
+        row_of[h][j] = 4 * ln + q;
+        act[h][j] = row_of[h][j] < a.rows;
+        any_r[h][j] = 4 * (16 * h + 8 * j) + q < a.rows;
+        lim[h][j] = act[h][j] ? min(n_tok, q_first + row_of[h][j] / a.G + 1) : n_tok;
+      }
     const int first_masked_tok = min(n_tok, q_first + 1);
-    float m_ref = -INFINITY;  // reference maximum (log2 units)
-    float l_run = 0.f;
+
+    float m_ref[H][2], l_run[H][2], m_g[H][2];
+    bool have_g[H][2];
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m_ref[h][j] = -INFINITY;
+        l_run[h][j] = 0.f;  // this thread's share (16 of the 64 columns of every tile)
+        m_g[h][j] = -INFINITY;
+        have_g[h][j] = false;
+      }
     bool failed = false;
 
-    for (int k = 0; k < my_tiles; ++k) {
+    // the split's partial slot of one of this thread's rows
+    auto dst_of = [&](int h, int j) -> float* {
+      const int r = row_of[h][j];
+      const size_t grow = (static_cast<size_t>(b) * a.num_q + r / a.G) * a.Hq + kvh * a.G + r % a.G;
+      return a.part_o + (grow * a.nsplit + split) * D;
+    };
+    auto o_addr = [&](int h, int cb) -> uint32_t {
+      return tmem_base + qlane + (static_cast<uint32_t>(16 * h) << 16) + kColO + 64 * cb;
+    };
+
+    // Page validity, once for the whole split: a tile with a page outside the
+    // pool is skipped (the producers load zeros for it and raise
+    // WMTP_DEV_PAGE_OOB).  In the common case every entry is valid and no tile
+    // needs a check; otherwise the tiles read their entries as they go.
+    {
+      const int box_rows = min(a.page_size, kTileTokens);
+      const int first = t_begin * kTileTokens, last = min(t_end * kTileTokens, n_tok);
+      bool ok = true;
+      for (int tok = first + (threadIdx.x - 64) * box_rows; tok < last; tok += 128 * box_rows) {
+        const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size];
+        ok = ok && pg >= 0 && pg < a.num_pages;
+      }
+      if (!__all_sync(0xffffffffu, ok) && lane == 0) *split_bad = 1;
+      ptx::named_bar_sync(kBarSoftmax, 128);
+    }
+    const bool split_ok = *split_bad == 0;
+
+    for (int k = 0; k < my_tiles && !failed; ++k) {
       const int sb = k & 1;
       // S(k) complete implies K(k) landed.  (The K ring itself is not waited
       // on here: its stage may already hold a later tile, so a parity wait on
       // it would be ambiguous.)
-      const bool ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8 * sb, (k >> 1) & 1, abort_flag));
-      if (!ok) {
+      if (!__all_sync(0xffffffffu, tc_wait(bar_s_full + 8 * sb, (k >> 1) & 1, abort_flag))) {
         failed = true;
-        break;  // this warp stops; the MMA warp times out or sees the abort
+        break;  // this warp stops; the MMA warps time out or see the abort
       }
       tc::fence_after_sync();
       const int tok0 = (t_begin + k) * kTileTokens;
-      // a tile with a page outside the pool is skipped (the producers loaded
-      // zeros for it and raised WMTP_DEV_PAGE_OOB)
-      bool tile_ok = true;
-      for (int tok = tok0; tok < min(tok0 + kTileTokens, n_tok); tok += min(a.page_size, kTileTokens)) {
-        const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size];
-        tile_ok = tile_ok && pg >= 0 && pg < a.num_pages;
-      }
-      const uint32_t s_addr = tmem_base + lane_addr + kColS + sb * 64;
-
-      uint32_t sraw[64];
-      tc::tmem_ld32(s_addr, sraw);
-      tc::tmem_ld32(s_addr + 32, sraw + 32);
-      float x[64];
-      float mx = -INFINITY;
-      if (tok0 + kTileTokens <= first_masked_tok) {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          x[j] = tile_ok ? __uint_as_float(sraw[j]) * a.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, x[j]);
-        }
-      } else {  // tile holding the causal tail and/or the end of the sequence
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int t = tok0 + j;
-          x[j] = (tile_ok && t < lim && t < n_tok) ? __uint_as_float(sraw[j]) * a.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, x[j]);
-        }
-      }
-      // raise the reference maximum only when the tile exceeds it by more
-      // than 2^8; rows whose reference moved rescale their O row and sum
-      float alpha = 1.f;
-      bool moved = false;
-      if (mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx != -INFINITY)) {
-        alpha = (m_ref == -INFINITY) ? 0.f : ptx::ex2(m_ref - mx);
-        moved = m_ref != -INFINITY;
-        m_ref = mx;
-      }
-      const float base = (m_ref == -INFINITY) ? 0.f : m_ref - kPShiftLog2;
-      if (__any_sync(0xffffffffu, moved)) {
-        // PV(k-1) must have finished before O is rewritten.  S(k) arriving
-        // implies PV(k-2) completed (issued before QK(k)), so the pending
-        // o_done phase is PV(k-1)'s and a parity wait is unambiguous.
+      const bool run_start = k > 0 && (k % kRunTiles) == 0;
+      bool o_ready = false;  // PV(k-1) known complete
+      if (run_start) {
+        // fold the finished run into the split's fp32 partial, in units of
+        // the current reference: G = G 2^(m_g - m_ref) + O; PV(k) then starts
+        // a fresh accumulation.  S(k) arriving implies PV(k-2) completed, so
+        // the pending o_done phase is PV(k-1)'s.
         if (!__all_sync(0xffffffffu, tc_wait(bar_o_done, (k - 1) & 1, abort_flag))) {
           failed = true;
           break;
         }
         tc::fence_after_sync();
-        const float f = moved ? alpha : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[32];
-          tc::tmem_ld32(tmem_base + lane_addr + kColO + 32 * c, o);
+        o_ready = true;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-          tc::tmem_st32(tmem_base + lane_addr + kColO + 32 * c, o);
+        for (int h = 0; h < H; ++h) {
+          if (!(any_r[h][0] || any_r[h][1])) continue;
+          float gs[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) gs[j] = have_g[h][j] ? ptx::ex2(m_g[h][j] - m_ref[h][j]) : 0.f;
+#pragma unroll 1
+          for (int cb = 0; cb < 4; ++cb) {
+            uint32_t o[32];
+            tc::tmem_ld_16x256b_x8(o_addr(h, cb), o);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              if (!act[h][j] || m_ref[h][j] == -INFINITY) continue;
+              float* d = dst_of(h, j) + 64 * cb + cq;
+#pragma unroll
+              for (int r = 0; r < 8; ++r) {
+                float2* g = reinterpret_cast<float2*>(d + 8 * r);
+                const float2 old = have_g[h][j] ? *g : make_float2(0.f, 0.f);
+                *g = make_float2(old.x * gs[j] + __uint_as_float(o[4 * r + 2 * j]),
+                                 old.y * gs[j] + __uint_as_float(o[4 * r + 2 * j + 1]));
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (m_ref[h][j] != -INFINITY) {
+              m_g[h][j] = m_ref[h][j];
+              have_g[h][j] = true;
+            }
         }
       }
-      // P = 2^(x - m_ref + 7) as fp16 pairs, back into the S columns
-      float sum = 0.f;
-      uint32_t ph[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float p0 = ptx::ex2(x[2 * j] - base);  // 2^-inf = 0 for masked entries
-        const float p1 = ptx::ex2(x[2 * j + 1] - base);
-        sum += p0 + p1;
-        ph[j] = ptx::pack_f16x2(p0, p1);
+      bool tile_ok = true;
+      if (!split_ok) {
+        for (int tok = tok0; tok < min(tok0 + kTileTokens, n_tok); tok += min(a.page_size, kTileTokens)) {
+          const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size];
+          tile_ok = tile_ok && pg >= 0 && pg < a.num_pages;
+        }
       }
-      l_run = l_run * alpha + sum;
-      tc::tmem_st32(s_addr, ph);
+      const bool masked_tile = tok0 + kTileTokens > first_masked_tok || !tile_ok;
+      // V rows past the end of the sequence hold stale pool bytes: zero them
+      // before PV reads the tile, so their 0 weights add exactly 0
+      if (tok0 + kTileTokens > n_tok) {
+        const int stage = k % VS;
+        if (!__all_sync(0xffffffffu, tc_wait(bar_v_full + 8 * stage, (k / VS) & 1, abort_flag))) {
+          failed = true;
+          break;
+        }
+        const int r0 = max(n_tok - tok0, 0);
+        const uint32_t vt = sbase + Plan::kOffV + stage * Plan::kTileBytes;
+        // 16-byte unit c (0..31) of token row r: chunk c / 8, unit c % 8 (a
+        // whole row is zeroed, so the swizzle does not matter)
+        for (int u = threadIdx.x - 64; u < (kTileTokens - r0) * 32; u += 128) {
+          const int r = r0 + u / 32, c = u % 32;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vt + (c >> 3) * Plan::kChunkBytes +
+                                                                       r * 128 + ((c & 7) << 4)),
+                       "r"(0)
+                       : "memory");
+        }
+        ptx::fence_proxy_async_smem();
+      }
+
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        const uint32_t s_addr = tmem_base + qlane + (static_cast<uint32_t>(16 * h) << 16) + kColS + sb * 64;
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ph[i] = pl[i] = 0u;
+        if (any_r[h][0] || any_r[h][1]) {
+          uint32_t sraw[32];
+          tc::tmem_ld_16x256b_x8(s_addr, sraw);
+          float x[2][16];
+          float mx[2] = {-INFINITY, -INFINITY};
+          // sub-row groups without any row are skipped (warp-uniform); a
+          // tile without masked positions takes the short path
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (!any_r[h][j]) continue;
+            if (!masked_tile) {
+#pragma unroll
+              for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  x[j][2 * r + e] = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
+                  mx[j] = fmaxf(mx[j], x[j][2 * r + e]);
+                }
+            } else {
+#pragma unroll
+              for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int t = tok0 + 8 * r + cq + e;
+                  const float s = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
+                  x[j][2 * r + e] = (tile_ok && t < lim[h][j] && t < n_tok) ? s : -INFINITY;
+                  mx[j] = fmaxf(mx[j], x[j][2 * r + e]);
+                }
+            }
+            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 1));
+            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 2));
+          }
+          // raise the reference maximum only when the tile exceeds it by more
+          // than 2^8; rows whose reference moved rescale their O row and sum
+          float alpha[2] = {1.f, 1.f};
+          bool moved = false;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (mx[j] > m_ref[h][j] + kRescaleLog2 || (m_ref[h][j] == -INFINITY && mx[j] != -INFINITY)) {
+              alpha[j] = (m_ref[h][j] == -INFINITY) ? 0.f : ptx::ex2(m_ref[h][j] - mx[j]);
+              moved = moved || m_ref[h][j] != -INFINITY;
+              m_ref[h][j] = mx[j];
+            }
+            l_run[h][j] *= alpha[j];
+          }
+          // a new run starts from an empty accumulator: nothing to rescale
+          if (!run_start && __any_sync(0xffffffffu, moved)) {
+            // PV(k-1) must have finished before O is rewritten.  S(k) arriving
+            // implies PV(k-2) completed (issued before QK(k)), so the pending
+            // o_done phase is PV(k-1)'s and a parity wait is unambiguous.
+            if (!o_ready) {
+              if (!__all_sync(0xffffffffu, tc_wait(bar_o_done, (k - 1) & 1, abort_flag))) {
+                failed = true;
+                break;
+              }
+              tc::fence_after_sync();
+              o_ready = true;
+            }
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+              uint32_t o[32];
+              tc::tmem_ld_16x256b_x8(o_addr(h, cb), o);
+#pragma unroll
+              for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                  for (int e = 0; e < 2; ++e)
+                    o[4 * r + 2 * j + e] = __float_as_uint(__uint_as_float(o[4 * r + 2 * j + e]) * alpha[j]);
+              tc::tmem_st_16x256b_x8(o_addr(h, cb), o);
+            }
+          }
+          // P = 2^(x - m_ref) as bf16 hi + lo pairs (token pair 4 r + lane % 4
+          // of the row), back into the S columns
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (!any_r[h][j]) continue;
+            const float base = (m_ref[h][j] == -INFINITY) ? 0.f : m_ref[h][j];
+            float sum = 0.f;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              const float p0 = ptx::ex2(x[j][2 * r] - base);  // 2^-inf = 0 for masked entries
+              const float p1 = ptx::ex2(x[j][2 * r + 1] - base);
+              sum += p0 + p1;
+              split_pack(p0, p1, ph[2 * r + j], pl[2 * r + j]);
+            }
+            l_run[h][j] += sum;
+          }
+        }
+        tc::tmem_st_16x128b_x8(s_addr, ph);
+        tc::tmem_st_16x128b_x8(s_addr + 32, pl);
+      }
+      if (failed) break;
 
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_p_full + 8 * sb);
     }
 
-    // ---- finish: normalised partial output and log-sum-exp of this row
+    // ---- finish: normalised partial output and log-sum-exp of each row
     if (!failed && my_tiles > 0) {
       // mma_final completes once, when every MMA of the CTA has completed (a
       // parity wait on o_done could not tell PV(n-2)'s phase from PV(n)'s
@@ -528,38 +676,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) set_status(a.status, kDevTimeout);
       *abort_flag = 1;
     }
-    const float inv = (l_run > 0.f && !failed) ? 1.f / l_run : 0.f;
-    const size_t grow =
-        row_active ? (static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G : 0;
-    float* dst = a.part_o + (grow * a.nsplit + split) * D;
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      float inv[2], gs[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        // the row's sum: each of its four threads holds a quarter
+        float l = l_run[h][j];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        l_run[h][j] = l;
+        inv[j] = (l > 0.f && !failed) ? 1.f / l : 0.f;
+        gs[j] = (have_g[h][j] && !failed) ? ptx::ex2(m_g[h][j] - m_ref[h][j]) : 0.f;
+      }
+      if (!(any_r[h][0] || any_r[h][1])) continue;
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {  // two 128-column TMEM loads per row
-      uint32_t o[128];
-      if (my_tiles > 0 && !failed) {
-        tc::tmem_ld128(tmem_base + lane_addr + kColO + 128 * c, o);
-      } else {
+      for (int cb = 0; cb < 4; ++cb) {
+        uint32_t o[32];
+        if (my_tiles > 0 && !failed) {
+          tc::tmem_ld_16x256b_x8(o_addr(h, cb), o);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 128; ++j) o[j] = 0u;
-      }
-      if (row_active) {
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
 #pragma unroll
-        for (int j = 0; j < 128; j += 4)
-          *reinterpret_cast<float4*>(dst + 128 * c + j) =
-              make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
-                          __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+        for (int j = 0; j < 2; ++j) {
+          if (!act[h][j]) continue;
+          float* d = dst_of(h, j) + 64 * cb + cq;
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            float2* g = reinterpret_cast<float2*>(d + 8 * r);
+            const float2 old = (have_g[h][j] && !failed) ? *g : make_float2(0.f, 0.f);
+            *g = make_float2((old.x * gs[j] + __uint_as_float(o[4 * r + 2 * j])) * inv[j],
+                             (old.y * gs[j] + __uint_as_float(o[4 * r + 2 * j + 1])) * inv[j]);
+          }
+        }
       }
-    }
-    if (row_active) {
-      // m_ref is in log2 units of the scaled score; l_run carries the 2^7
-      // offset of P
-      a.part_lse[grow * a.nsplit + split] =
-          (l_run > 0.f && !failed) ? (m_ref - kPShiftLog2) * 0.69314718055994531f + logf(l_run) : -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        if (act[h][j] && (lane & 3) == 0) {
+          const int r = row_of[h][j];
+          const size_t grow = (static_cast<size_t>(b) * a.num_q + r / a.G) * a.Hq + kvh * a.G + r % a.G;
+          // m_ref is in log2 units of the scaled score
+          a.part_lse[grow * a.nsplit + split] = (l_run[h][j] > 0.f && !failed)
+                                                    ? m_ref[h][j] * 0.69314718055994531f + logf(l_run[h][j])
+                                                    : -INFINITY;
+        }
+      }
     }
     tc::fence_before_sync();
   }
 
-  // ---- every MMA has completed (the MMA lane waited for its final commit);
-  // free the tensor memory
+  // ---- every MMA has completed (the MMA lanes waited for their final
+  // commit); free the tensor memory
   ptx::named_bar_sync(kBarTmem, 160);
   if (warp == 1) {
     tc::fence_after_sync();

@@ -418,14 +418,64 @@ def test_workspace_query_matches_binding():
     assert w.workspace_bytes("verify", p, 1, num_q=4, max_pages=16384) >= n
 
 
-def test_verify_flags_values_beyond_fp16_range():
-    """The verify value product runs in fp16; a V value of 2^16 or more must
-    raise the range bit instead of passing silently."""
+def test_verify_takes_values_of_any_bf16_magnitude():
+    """The tcgen05 verify reads V in its own bf16 format: values far beyond
+    the fp16 range (1e5, -3e30) and tiny ones (1e-30) go through exactly, and
+    no status bit is raised."""
     p = _params(16, 2, 256, 64)
     kv = _paged(95, 1, 2, 256, 64, [300])
     kv.v_pool[kv.page_table[0, 1], 1, 5, 7] = 1.0e5
+    kv.v_pool[kv.page_table[0, 2], 0, 9, 100] = -3.0e30
+    kv.v_pool[kv.page_table[0, 0], 1, 0, :] = 1.0e-30
     q = synth.queries(96, (1, 4, 16, 256), device=DEV)
     status = w.new_status(DEV)
-    w.verify_attn(p, q, cache_of(kv), status=status)
+    out, lse = w.verify_attn(p, q, cache_of(kv), status=status)
     torch.cuda.synchronize()
-    assert int(status.item()) & L.DEV_V_RANGE
+    assert int(status.item()) == 0
+    kp, vp, pt, ln = _oracle_pools(kv)
+    ref, ref_lse = oracle.verify_attn(f64(q), kp, vp, pt, ln, 64, 1 / 16)
+    # relative to each element's own scale: the planted values dominate a few
+    # output columns by 30 orders of magnitude
+    got = f64(out)
+    scale = np.maximum(np.abs(ref), 1.0)
+    assert np.all(np.abs(got - ref) <= 2e-3 * scale), float(np.max(np.abs(got - ref) / scale))
+    assert_lse_close(f64(lse), ref_lse, "verify large values")
+
+
+@pytest.mark.parametrize("kind", ["verify", "draft"])
+def test_page_outside_the_pool_is_skipped(kind):
+    """A page-table entry outside the pool raises WMTP_DEV_PAGE_OOB and the
+    tile holding it is left out of the attention: the result equals the
+    oracle's attention over the other positions (head_dim 256, page 64, so
+    one page is one 64-token tile; verify runs on the tcgen05 kernel)."""
+    Hkv, G, D, P = 2, 8, 256, 64
+    num_q = 4 if kind == "verify" else 1
+    n = 9000 + num_q
+    p = _params(G * Hkv, Hkv, D, P)
+    kv = _paged(97, 1, Hkv, D, P, [n])
+    bad_page = 37  # positions 2368 .. 2431
+    kv.page_table[0, bad_page] = kv.k_pool.shape[0] + 5
+    shape = (1, num_q, G * Hkv, D) if kind == "verify" else (1, G * Hkv, D)
+    q = synth.queries(98, shape, device=DEV)
+    status = w.new_status(DEV)
+    fn = w.verify_attn if kind == "verify" else w.draft_attn_full
+    out, lse = fn(p, q, cache_of(kv), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & L.DEV_PAGE_OOB
+    # the oracle over every position but the bad page's, gathered through the
+    # valid entries of the table
+    kp, vp = f64(kv.k_pool), f64(kv.v_pool)
+    pt = kv.page_table.cpu().numpy()[0].astype(np.int64)
+    keep = np.array([t for t in range(n) if t // P != bad_page])
+    qs = f64(q).reshape(num_q, G * Hkv, D)
+    got, got_lse = f64(out).reshape(num_q, G * Hkv, D), f64(lse).reshape(num_q, G * Hkv)
+    for kvh in range(Hkv):
+        K = kp[pt[keep // P], kvh, keep % P]
+        V = vp[pt[keep // P], kvh, keep % P]
+        for i in range(num_q):
+            last = n - num_q + i  # causal limit of query i
+            sel = keep <= last
+            rows = slice(kvh * G, (kvh + 1) * G)
+            ref, ref_lse = oracle.attend_rows(qs[i, rows], K[sel], V[sel], 1 / 16)
+            assert_close(got[i, rows], ref, f"{kind} skip kvh {kvh} q {i}")
+            assert_lse_close(got_lse[i, rows], ref_lse, f"{kind} skip kvh {kvh} q {i}")

@@ -1,5 +1,5 @@
-"""GPU parity of the tcgen05 verify kernel on the inputs that reach its
-hardest numerics, against the fp64 oracle.
+"""GPU parity of the attention kernels on the inputs that reach their
+hardest numerics, against the fp64 oracle (mostly the tcgen05 verify).
 
 The verify kernel keeps a per-row reference maximum that it raises only when
 a tile beats it by more than 2^8, and then rescales that row of the
@@ -21,6 +21,8 @@ that do.
   the kernel keeps them in the normal range.
 * A planted key among the new tokens is seen only by the queries at or after
   its position (causal limit on the last tile).
+* A flat sea of a million keys in one split (native draft, 64 sequences): an
+  accumulation of a million nearly equal products of one sign.
 
 The attention definition is the pages' (arxivlens view, Abstract: verification
 stays full-context); the oracle is plain fp64 softmax attention.
@@ -223,3 +225,44 @@ def test_verify_sink_over_a_flat_sea():
         assert_close(got, np.broadcast_to(ref, got.shape), f"sink over a flat sea kvh {kvh}")
         for b in range(B):
             assert_lse_close(got_lse[b], ref_lse, f"sink over a flat sea kvh {kvh} seq {b}")
+
+
+@pytest.mark.timeout(900)
+def test_native_draft_flat_sea_in_one_long_split():
+    """The native draft of 64 sequences of 1,048,576 tokens runs one split per
+    sequence and KV head, so one CTA accumulates a whole million-token
+    context.  With nearly equal weights and values of one sign (mean 2) an
+    accumulation that drops the low-order bits of each product against the
+    running sum would bias the result by ~0.5%; the kernel's runs of 8,192
+    tokens keep it inside the parity bar."""
+    G, Hkv, D, P, B = 8, 2, 256, 64, 64
+    Hq = G * Hkv
+    n = 1 << 20
+    npg = n // P
+    num_pages = 65
+    gen = torch.Generator(device=DEV).manual_seed(460)
+    k_pool = (torch.randn(num_pages, Hkv, P, D, generator=gen, device=DEV) * 1e-3).to(torch.bfloat16)
+    v_pool = (2.0 + 0.1 * torch.randn(num_pages, Hkv, P, D, generator=gen, device=DEV)).to(torch.bfloat16)
+    row = torch.arange(npg, dtype=torch.int32) % num_pages
+    kv = synth.PagedKV(k_pool, v_pool, row[None].expand(B, npg).contiguous().to(DEV),
+                       torch.full((B,), n, dtype=torch.int32, device=DEV), P)
+    q0 = synth.queries(461, (Hq, D), device=DEV)
+    q = q0[None].expand(B, Hq, D).contiguous()
+    p = w.params(Hq, Hkv, D, page_size=P)
+    status = w.new_status(DEV)
+    out, lse = w.draft_attn_full(p, q, cache_of(kv), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    tbl = row.numpy().astype(np.int64)
+    pos = np.arange(n)
+    kp, vp = f64(k_pool), f64(v_pool)
+    for kvh in range(Hkv):
+        K = kp[tbl[pos // P], kvh, pos % P]
+        V = vp[tbl[pos // P], kvh, pos % P]
+        rows = slice(kvh * G, (kvh + 1) * G)
+        ref, ref_lse = oracle.attend_prefixes(f64(q0[rows]), K, V, np.full(G, n), 1 / 16)
+        del K, V
+        got = f64(out[:, rows])
+        assert_close(got, np.broadcast_to(ref, got.shape), f"native draft flat sea kvh {kvh}")
+        for b in range(0, B, 21):
+            assert_lse_close(f64(lse[b, rows]), ref_lse, f"native draft flat sea kvh {kvh} seq {b}")
