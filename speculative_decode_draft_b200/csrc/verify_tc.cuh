@@ -10,12 +10,16 @@
 // the rows as the MMA M dimension (padded to M = 64, or to M = 128 for blocks
 // of 65..128 rows such as gamma = 8 with G = 8) and everything but K and V
 // kept in tensor memory (512 columns; the M=64 layout uses lanes 0..15 of
-// each of the four lane quadrants, M=128 all 32):
-//   columns   0..127  Q            bf16 pairs, the A operand of S = Q K^T
-//   columns 128..255  S / P x 2    fp32 scores of a tile; after the softmax
-//                                  columns 0..31 of the buffer hold P_hi and
-//                                  32..63 P_lo as bf16 pairs (P = hi + lo)
-//   columns 256..511  O            fp32 output accumulator, 256 head dims
+// each of the four lane quadrants, M=128 all 32).  For M = 64, Q sits in
+// shared memory and the scores have three TMEM buffers; for M = 128 (Q is
+// twice as large) Q sits in TMEM and the scores have two:
+//   M = 64:  columns 0..191 S / P x 3, columns 256..511 O
+//   M = 128: columns 0..127 Q (bf16 pairs), 128..255 S / P x 2, 256..511 O
+// An S buffer holds a tile's fp32 scores; after the softmax its columns 0..31
+// hold P_hi and 32..63 P_lo as bf16 pairs (P = hi + lo).  O is the fp32
+// output accumulator, 256 head dims.  QK(k) may overwrite buffer k % NB only
+// once PV(k - NB) has read it, so with three buffers the QK of a tile no
+// longer waits for the PV of the tile just before the previous one.
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
 // 16 (r % 4) + r / 4 for M=64, 32 (r % 4) + r / 4 for M=128), so the rows
 // spread over the four lane quadrants and each softmax warp owns a quarter of
@@ -79,21 +83,22 @@ constexpr int kVWarp = 7;
 constexpr int kBarTmem = 3;           // named barrier: QK issuer + softmax warps
 constexpr int kBarSoftmax = 4;        // named barrier: the softmax warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQ = 0;
-constexpr uint32_t kColS = 128;
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.f;   // lazy rescale threshold (log2 units)
 
-template <int KS, int VS>
+// QS: Q in shared memory (three score buffers) or in TMEM (two).
+template <int KS, int VS, bool QS>
 struct TcPlan {
-  static constexpr int kChunkBytes = 64 * 128;           // 64 tokens x 128 B
-  static constexpr int kTileBytes = 4 * kChunkBytes;      // one K or V tile, D = 256
+  static constexpr int kNB = QS ? 3 : 2;                  // S / P buffers in TMEM
+  static constexpr int kChunkBytes = 64 * 128;           // 64 tokens (or rows) x 128 B
+  static constexpr int kTileBytes = 4 * kChunkBytes;      // one K or V tile (or Q), D = 256
   static constexpr int kOffK = 0;                         // K ring: KS tiles
   static constexpr int kOffV = KS * kTileBytes;           // V ring: VS tiles
-  static constexpr int kOffBar = (KS + VS) * kTileBytes;
-  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
-  // o_done, mma_final, q_ready, pv_done[2]
-  static constexpr int kNumBars = 2 * KS + 2 * VS + 9;
+  static constexpr int kOffQ = (KS + VS) * kTileBytes;    // Q (QS only), 64 rows, K-major, 128-byte swizzle
+  static constexpr int kOffBar = kOffQ + (QS ? kTileBytes : 0);
+  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NB], p_full[NB],
+  // pv_done[NB], mma_final, q_ready
+  static constexpr int kNumBars = 2 * KS + 2 * VS + 3 * kNB + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, split page validity
   static constexpr int kBytes = kOffMisc + 12;
   static constexpr int kAlloc = kBytes + 1024;
@@ -121,12 +126,17 @@ __device__ __forceinline__ void split_pack(float p0, float p1, uint32_t& hi, uin
   lo = ptx::pack_bf16x2(p0 - ptx::bf16lo_to_f32(hi), p1 - ptx::bf16hi_to_f32(hi));
 }
 
-// M: MMA rows (64 or 128); the block's rows must not exceed it.
+// M: MMA rows (64 or 128); the block's rows must not exceed it.  M = 64
+// keeps Q in shared memory and three score buffers, M = 128 Q in TMEM and two.
 template <int KS, int VS, int M>
 __global__ void __launch_bounds__(kTcThreads, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const DecodeArgs a) {
-  using Plan = TcPlan<KS, VS>;
+  constexpr bool QS = M == 64;
+  using Plan = TcPlan<KS, VS, QS>;
+  constexpr int NB = Plan::kNB;
+  constexpr uint32_t kColQ = 0;            // TMEM Q (M = 128)
+  constexpr uint32_t kColS = QS ? 0 : 128;  // first score buffer
   constexpr int D = 256;
   static_assert(M == 64 || M == 128, "MMA rows: 64 or 128");
   constexpr int H = M / 64;  // sixteen-lane halves of a quadrant that hold rows
@@ -140,12 +150,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_k_empty = bar_k_full + 8 * KS;
   const uint32_t bar_v_full = bar_k_empty + 8 * KS;
   const uint32_t bar_v_empty = bar_v_full + 8 * VS;
-  const uint32_t bar_s_full = bar_v_empty + 8 * VS;
-  const uint32_t bar_p_full = bar_s_full + 16;
-  const uint32_t bar_o_done = bar_p_full + 16;
-  const uint32_t bar_final = bar_o_done + 8;
+  const uint32_t bar_s_full = bar_v_empty + 8 * VS;  // [NB]
+  const uint32_t bar_p_full = bar_s_full + 8 * NB;    // [NB]
+  const uint32_t bar_pv_done = bar_p_full + 8 * NB;   // [NB]: PV of the tiles using S/P buffer b
+  const uint32_t bar_final = bar_pv_done + 8 * NB;
   const uint32_t bar_q_ready = bar_final + 8;
-  const uint32_t bar_pv_done = bar_q_ready + 8;  // [2]: PV of the tiles using S/P buffer 0 / 1
   volatile int* split_bad = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
@@ -166,14 +175,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::mbar_init(bar_v_full + 8 * s, 1);
       ptx::mbar_init(bar_v_empty + 8 * s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NB; ++i) {
       ptx::mbar_init(bar_s_full + 8 * i, 1);
       ptx::mbar_init(bar_p_full + 8 * i, 4);
+      ptx::mbar_init(bar_pv_done + 8 * i, 1);
     }
-    ptx::mbar_init(bar_o_done, 1);
     ptx::mbar_init(bar_final, 2);  // one commit from each MMA-issuing lane
-    ptx::mbar_init(bar_pv_done, 1);
-    ptx::mbar_init(bar_pv_done + 8, 1);
     ptx::mbar_init(bar_q_ready, 4);
     *abort_flag = 0;
     *split_bad = 0;
@@ -309,12 +316,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t v_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffV, Plan::kChunkBytes, 1024);
       bool ok = true;
       for (int k = 0; ok && k < my_tiles; ++k) {
-        ok = tc_wait(bar_p_full + 8 * (k & 1), (k >> 1) & 1, abort_flag) &&
+        ok = tc_wait(bar_p_full + 8 * (k % NB), (k / NB) & 1, abort_flag) &&
              tc_wait(bar_v_full + 8 * (k % VS), (k / VS) & 1, abort_flag);
         if (!ok) break;
         tc::fence_after_sync();
         const uint64_t vd = v_desc0 + (static_cast<uint64_t>((k % VS) * Plan::kTileBytes) >> 4);
-        const uint32_t p_tmem = tmem_base + kColS + (k & 1) * 64;
+        const uint32_t p_tmem = tmem_base + kColS + (k % NB) * 64;
         const uint32_t fresh = (k % kRunTiles) == 0 ? 0u : 1u;  // 0: overwrite O
 #pragma unroll
         for (int kk = 0; kk < kTileTokens / 16; ++kk) {
@@ -324,8 +331,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc::mma_ts(tmem_base + kColO, p_tmem + 32 + 8 * kk, bd, kIdescPV, 1u);
         }
         tc::commit(bar_v_empty + 8 * (k % VS));
-        tc::commit(bar_o_done);
-        tc::commit(bar_pv_done + 8 * (k & 1));
+        tc::commit(bar_pv_done + 8 * (k % NB));
       }
       if (!ok) {
         if (*abort_flag == 0) set_status(a.status, kDevTimeout);
@@ -343,28 +349,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0 && my_tiles > 0) {
       // M = 64 whenever the rows fit: an M=64 MMA costs the same issue time
       // as M=128 for half the tensor work (and power)
-      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(M, 64, 0, 0);     // A (Q, TMEM), B (K) K-major
+      constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(M, 64, 0, 0);     // A (Q), B (K) K-major
       // descriptor start addresses are in 16-byte units in the low bits, so
       // moving an operand by n bytes adds n >> 4 to the descriptor
       const uint64_t k_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffK, 16, 1024);
+      const uint64_t q_desc0 = tc::smem_desc_sw128(sbase + Plan::kOffQ, 16, 1024);  // QS only
       // Q is staged into TMEM by the softmax warps while the first K/V tiles
       // are in flight
       bool ok = tc_wait(bar_q_ready, 0, abort_flag);
       for (int k = 0; ok && k < my_tiles; ++k) {
-        // S/P buffer k & 1 last held P(k-2): PV(k-2), issued by the other
+        // S/P buffer k % NB last held P(k-NB): PV(k-NB), issued by the other
         // lane, must have completed (its phase of pv_done; the next phase
         // needs P(k), which needs this S)
-        if (k >= 2 && !(ok = tc_wait(bar_pv_done + 8 * (k & 1), ((k - 2) >> 1) & 1, abort_flag))) break;
+        if (k >= NB && !(ok = tc_wait(bar_pv_done + 8 * (k % NB), ((k - NB) / NB) & 1, abort_flag))) break;
         if (!(ok = tc_wait(bar_k_full + 8 * (k % KS), (k / KS) & 1, abort_flag))) break;
         tc::fence_after_sync();
         const uint64_t kd = k_desc0 + (static_cast<uint64_t>((k % KS) * Plan::kTileBytes) >> 4);
-        const uint32_t d_tmem = tmem_base + kColS + (k & 1) * 64;
+        const uint32_t d_tmem = tmem_base + kColS + (k % NB) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * Plan::kChunkBytes + (kk & 3) * 32;
-          tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+          if constexpr (QS)
+            tc::mma_ss(d_tmem, q_desc0 + (ka >> 4), kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+          else
+            tc::mma_ts(d_tmem, tmem_base + kColQ + 8 * kk, kd + (ka >> 4), kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc::commit(bar_s_full + 8 * (k & 1));
+        tc::commit(bar_s_full + 8 * (k % NB));
         tc::commit(bar_k_empty + 8 * (k % KS));
       }
       if (!ok) {
@@ -382,8 +392,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp & 3;  // this warp's TMEM lane quadrant
     const uint32_t qlane = static_cast<uint32_t>(32 * q) << 16;
     {
-      // Q: thread `lane` stages row 4 lane + q into TMEM lane 32 q + lane
-      // (columns 0..127, bf16 pairs), zeros for padding rows; every load is
+      // Q: thread `lane` stages row 4 lane + q, MMA row 16 q + lane (M = 64)
+      // or 32 q + lane (M = 128), zeros for padding rows; every load is
       // issued before the first store so the row costs one global round trip
       const int row = 4 * lane + q;
       const bool q_active = lane < M / 4 && row < a.rows;
@@ -394,19 +404,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int j = 0; j < D / 8; ++j)
         v[j] = q_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
+      if constexpr (QS) {
+        // shared memory, K-major with the 128-byte swizzle the K tiles have:
+        // chunk c (head dims 64 c .. 64 c + 63) of MMA row m at c * 8 KB + 128 m,
+        // 16-byte unit u at position u ^ (m % 8)
+        if (lane < 16) {
+          const int m = 16 * q + lane;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t wq[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          wq[4 * j] = v[8 * c + j].x;
-          wq[4 * j + 1] = v[8 * c + j].y;
-          wq[4 * j + 2] = v[8 * c + j].z;
-          wq[4 * j + 3] = v[8 * c + j].w;
+          for (int j = 0; j < D / 8; ++j) {
+            const uint32_t dst = sbase + Plan::kOffQ + (j >> 3) * Plan::kChunkBytes + m * 128 +
+                                 (((j & 7) ^ (m & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[j].x), "r"(v[j].y),
+                         "r"(v[j].z), "r"(v[j].w)
+                         : "memory");
+          }
         }
-        tc::tmem_st32(tmem_base + qlane + kColQ + 32 * c, wq);
+        ptx::fence_proxy_async_smem();  // generic writes before the tensor core reads
+      } else {
+        // TMEM lane 32 q + lane, columns 0..127 (bf16 pairs)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t wq[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            wq[4 * j] = v[8 * c + j].x;
+            wq[4 * j + 1] = v[8 * c + j].y;
+            wq[4 * j + 2] = v[8 * c + j].z;
+            wq[4 * j + 3] = v[8 * c + j].w;
+          }
+          tc::tmem_st32(tmem_base + qlane + kColQ + 32 * c, wq);
+        }
+        tc::fence_before_sync();
       }
-      tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_q_ready);
     }
@@ -474,11 +503,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool split_ok = *split_bad == 0;
 
     for (int k = 0; k < my_tiles && !failed; ++k) {
-      const int sb = k & 1;
+      const int sb = k % NB;
       // S(k) complete implies K(k) landed.  (The K ring itself is not waited
       // on here: its stage may already hold a later tile, so a parity wait on
       // it would be ambiguous.)
-      if (!__all_sync(0xffffffffu, tc_wait(bar_s_full + 8 * sb, (k >> 1) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, tc_wait(bar_s_full + 8 * sb, (k / NB) & 1, abort_flag))) {
         failed = true;
         break;  // this warp stops; the MMA warps time out or see the abort
       }
@@ -489,9 +518,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (run_start) {
         // fold the finished run into the split's fp32 partial, in units of
         // the current reference: G = G 2^(m_g - m_ref) + O; PV(k) then starts
-        // a fresh accumulation.  S(k) arriving implies PV(k-2) completed, so
-        // the pending o_done phase is PV(k-1)'s.
-        if (!__all_sync(0xffffffffu, tc_wait(bar_o_done, (k - 1) & 1, abort_flag))) {
+        // a fresh accumulation.  PV(k-1) completes the pv_done phase of its
+        // buffer; the buffer's next phase needs P(k-1+NB), so the wait is
+        // unambiguous.
+        if (!__all_sync(0xffffffffu, tc_wait(bar_pv_done + 8 * ((k - 1) % NB), ((k - 1) / NB) & 1, abort_flag))) {
           failed = true;
           break;
         }
@@ -578,10 +608,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
               for (int r = 0; r < 8; ++r)
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
+                for (int e = 0; e < 2; ++e)
                   x[j][2 * r + e] = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
-                  mx[j] = fmaxf(mx[j], x[j][2 * r + e]);
-                }
             } else {
 #pragma unroll
               for (int r = 0; r < 8; ++r)
@@ -590,9 +618,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                   const int t = tok0 + 8 * r + cq + e;
                   const float s = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
                   x[j][2 * r + e] = (tile_ok && t < lim[h][j] && t < n_tok) ? s : -INFINITY;
-                  mx[j] = fmaxf(mx[j], x[j][2 * r + e]);
                 }
             }
+            // pairwise maximum (a tree keeps the dependent chain short)
+            float t8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t8[i] = fmaxf(x[j][2 * i], x[j][2 * i + 1]);
+#pragma unroll
+            for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+              for (int i = 0; i < w2; ++i) t8[i] = fmaxf(t8[i], t8[i + w2]);
+            mx[j] = t8[0];
             mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 1));
             mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 2));
           }
@@ -611,11 +647,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           // a new run starts from an empty accumulator: nothing to rescale
           if (!run_start && __any_sync(0xffffffffu, moved)) {
-            // PV(k-1) must have finished before O is rewritten.  S(k) arriving
-            // implies PV(k-2) completed (issued before QK(k)), so the pending
-            // o_done phase is PV(k-1)'s and a parity wait is unambiguous.
+            // PV(k-1) must have finished before O is rewritten (the pv_done
+            // phase of its buffer, as for the fold above)
             if (!o_ready) {
-              if (!__all_sync(0xffffffffu, tc_wait(bar_o_done, (k - 1) & 1, abort_flag))) {
+              if (!__all_sync(0xffffffffu, tc_wait(bar_pv_done + 8 * ((k - 1) % NB), ((k - 1) / NB) & 1,
+                                                   abort_flag))) {
                 failed = true;
                 break;
               }
@@ -642,15 +678,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int j = 0; j < 2; ++j) {
             if (!any_r[h][j]) continue;
             const float base = (m_ref[h][j] == -INFINITY) ? 0.f : m_ref[h][j];
-            float sum = 0.f;
+            float ps[8];
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
               const float p0 = ptx::ex2(x[j][2 * r] - base);  // 2^-inf = 0 for masked entries
               const float p1 = ptx::ex2(x[j][2 * r + 1] - base);
-              sum += p0 + p1;
+              ps[r] = p0 + p1;
               split_pack(p0, p1, ph[2 * r + j], pl[2 * r + j]);
             }
-            l_run[h][j] += sum;
+#pragma unroll
+            for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+              for (int i = 0; i < w2; ++i) ps[i] += ps[i + w2];
+            l_run[h][j] += ps[0];
           }
         }
         tc::tmem_st_16x128b_x8(s_addr, ph);
@@ -665,9 +705,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     // ---- finish: normalised partial output and log-sum-exp of each row
     if (!failed && my_tiles > 0) {
-      // mma_final completes once, when every MMA of the CTA has completed (a
-      // parity wait on o_done could not tell PV(n-2)'s phase from PV(n)'s
-      // once both PV(n-2) and PV(n-1) have completed)
+      // mma_final completes once, when every MMA of the CTA has completed
       if (!__all_sync(0xffffffffu, tc_wait(bar_final, 0, abort_flag))) failed = true;
       tc::fence_after_sync();
     }

@@ -255,7 +255,7 @@ wmtp_status launch_decode(int D, int NT, const CUtensorMap& tk, const CUtensorMa
 template <int M>
 wmtp_status launch_verify_tc_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int B,
                                cudaStream_t st) {
-  constexpr int alloc = TcPlan<kTcKStages, kTcVStages>::kAlloc;
+  constexpr int alloc = TcPlan<kTcKStages, kTcVStages, M == 64>::kAlloc;
   static_assert(alloc <= kSmemLimit, "shared-memory plan exceeds the sm_100 per-block limit");
   auto kern = verify_tc_kernel<kTcKStages, kTcVStages, M>;
   static SmemAttrOnce once;
