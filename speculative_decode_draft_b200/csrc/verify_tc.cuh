@@ -166,14 +166,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- set-up: barriers and tensor memory
+  // each producer initialises its own ring's barriers, so it can issue its
+  // first load before the block-wide barrier below
+  if (threadIdx.x == kVWarp * 32) {
+    for (int s = 0; s < VS; ++s) {
+      ptx::mbar_init(bar_v_full + 8 * s, 1);
+      ptx::mbar_init(bar_v_empty + 8 * s, 1);
+    }
+    ptx::fence_mbar_init();
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < KS; ++s) {
       ptx::mbar_init(bar_k_full + 8 * s, 1);
       ptx::mbar_init(bar_k_empty + 8 * s, 1);
-    }
-    for (int s = 0; s < VS; ++s) {
-      ptx::mbar_init(bar_v_full + 8 * s, 1);
-      ptx::mbar_init(bar_v_empty + 8 * s, 1);
     }
     for (int i = 0; i < NB; ++i) {
       ptx::mbar_init(bar_s_full + 8 * i, 1);
@@ -193,6 +198,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // every global-memory access comes after this: with a programmatic launch
   // the set-up above overlaps the previous kernel's tail
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // ---- Q first: the softmax warps' loads leave before any K/V load of the
+  // CTA.  Thread `lane` of softmax warp q holds row 4 lane + q (zeros for
+  // padding rows); every load is issued before the first use.
+  const int q = warp & 3;  // the TMEM lane quadrant of a softmax warp
+  const bool softmax_warp = warp >= 2 && warp < 6;
+  uint4 qv[D / 8];
+  if (softmax_warp) {
+    const int row = 4 * lane + q;
+    const bool q_active = lane < M / 4 && row < a.rows;
+    const __nv_bfloat16* src =
+        q_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
+                 : nullptr;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j)
+      qv[j] = q_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
+  }
+  // the page-table entries of this split's first tiles, guessed from the
+  // cache's capacity (exact when the sequence fills it), head for L2 while
+  // kv_len is read
+  if (warp == 0 && lane < KS) {
+    const int nt_cap = (a.max_pages * a.page_size + kTileTokens - 1) / kTileTokens;
+    const int t = split * ((nt_cap + a.nsplit - 1) / a.nsplit) + lane;
+    if (t < nt_cap)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a.page_table + static_cast<size_t>(b) * a.max_pages +
+                                                        (t * kTileTokens) / a.page_size));
+  }
   // ---- token range of this split
   int n_tok = a.kv_len[b];
   if (n_tok != 0 &&
@@ -255,12 +286,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::tma_load_3d(dst + c * Plan::kChunkBytes + j * box_rows * 128, tmap, fb, c * 64, ys[j], zs[j], pol);
     }
   };
-  // start the page-table reads of the first tiles now; the producers' own
-  // loads then hit L2
-  if (warp == 0 && lane < VS && lane < my_tiles) {
+  // tile 0 of each ring goes out before the block-wide barrier (the
+  // producers initialised their own barriers), and the page-table lines of
+  // the next tiles head for L2
+  int issued_pre = 0;
+  if ((warp == 0 || warp == kVWarp) && lane == 0 && my_tiles > 0) {
+    ptx::prefetch_tmap(tmap);
+    int pg0[4];
+    pages_of(0, pg0);
+    produce(0, pg0, ptx::policy_evict_first());
+    issued_pre = 1;
+  }
+  if (warp == 0 && lane >= 1 && lane <= VS && lane < my_tiles) {
     const int* pte = a.page_table + static_cast<size_t>(b) * a.max_pages +
                      ((t_begin + lane) * kTileTokens) / a.page_size;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(pte));
+  }
+  // Q of M = 64 goes to shared memory now (K-major with the 128-byte swizzle
+  // the K tiles have: chunk c (head dims 64 c .. 64 c + 63) of MMA row m at
+  // c * 8 KB + 128 m, 16-byte unit u at position u ^ (m % 8))
+  if constexpr (QS) {
+    if (softmax_warp && lane < 16) {
+      const int m = 16 * q + lane;
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) {
+        const uint32_t dst = sbase + Plan::kOffQ + (j >> 3) * Plan::kChunkBytes + m * 128 + (((j & 7) ^ (m & 7)) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(qv[j].x), "r"(qv[j].y),
+                     "r"(qv[j].z), "r"(qv[j].w)
+                     : "memory");
+      }
+    }
+    if (softmax_warp) ptx::fence_proxy_async_smem();  // generic writes before the tensor core reads
   }
 
   tc::fence_before_sync();
@@ -273,12 +329,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // =================================================================== producers
   if (warp == 0 || warp == kVWarp) {
     if (lane == 0 && my_tiles > 0) {
-      ptx::prefetch_tmap(tmap);
       const uint64_t pol = ptx::policy_evict_first();
-      int issued = 0;
+      int issued = issued_pre;
       int pg_cur[4], pg_nxt[4];
-      pages_of(0, pg_cur);
-      for (int k = 0; k < my_tiles; ++k) {
+      pages_of(issued, pg_cur);
+      for (int k = issued; k < my_tiles; ++k) {
         // entries four tiles ahead head for L2; the next tile's are read now
         const int ahead = (t_begin + k + 4) * kTileTokens;
         if (k + 4 < my_tiles && ahead < n_tok)
@@ -389,48 +444,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ================================================================= softmax
-    const int q = warp & 3;  // this warp's TMEM lane quadrant
     const uint32_t qlane = static_cast<uint32_t>(32 * q) << 16;
     {
-      // Q: thread `lane` stages row 4 lane + q, MMA row 16 q + lane (M = 64)
-      // or 32 q + lane (M = 128), zeros for padding rows; every load is
-      // issued before the first store so the row costs one global round trip
-      const int row = 4 * lane + q;
-      const bool q_active = lane < M / 4 && row < a.rows;
-      const __nv_bfloat16* src =
-          q_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
-                   : nullptr;
-      uint4 v[D / 8];
-#pragma unroll
-      for (int j = 0; j < D / 8; ++j)
-        v[j] = q_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
-      if constexpr (QS) {
-        // shared memory, K-major with the 128-byte swizzle the K tiles have:
-        // chunk c (head dims 64 c .. 64 c + 63) of MMA row m at c * 8 KB + 128 m,
-        // 16-byte unit u at position u ^ (m % 8)
-        if (lane < 16) {
-          const int m = 16 * q + lane;
-#pragma unroll
-          for (int j = 0; j < D / 8; ++j) {
-            const uint32_t dst = sbase + Plan::kOffQ + (j >> 3) * Plan::kChunkBytes + m * 128 +
-                                 (((j & 7) ^ (m & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[j].x), "r"(v[j].y),
-                         "r"(v[j].z), "r"(v[j].w)
-                         : "memory");
-          }
-        }
-        ptx::fence_proxy_async_smem();  // generic writes before the tensor core reads
-      } else {
-        // TMEM lane 32 q + lane, columns 0..127 (bf16 pairs)
+      // Q of M = 128 goes into TMEM lane 32 q + lane, columns 0..127 (bf16
+      // pairs); Q of M = 64 is already in shared memory
+      if constexpr (!QS) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t wq[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            wq[4 * j] = v[8 * c + j].x;
-            wq[4 * j + 1] = v[8 * c + j].y;
-            wq[4 * j + 2] = v[8 * c + j].z;
-            wq[4 * j + 3] = v[8 * c + j].w;
+            wq[4 * j] = qv[8 * c + j].x;
+            wq[4 * j + 1] = qv[8 * c + j].y;
+            wq[4 * j + 2] = qv[8 * c + j].z;
+            wq[4 * j + 3] = qv[8 * c + j].w;
           }
           tc::tmem_st32(tmem_base + qlane + kColQ + 32 * c, wq);
         }
