@@ -569,20 +569,24 @@ def cores_used():
     return len(os.sched_getaffinity(0))
 
 
-# DRAM traffic of one verify_tc_kernel launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) from one ncu capture on the 128K workload (a few GB
-# on the device), with the K/V tokens that launch read.  The traffic of a
-# launch grows in proportion to the tokens it reads (every K/V byte crosses
-# HBM once; the partials are a few MB), so it is scaled by tokens to the
-# bench's workload.  It is reported only while the kernel's code (its sources
-# with comments and whitespace removed) hashes to the value it was captured
-# on; otherwise roofline.traffic is null.
+# DRAM traffic of one verify_tc_kernel launch from one ncu capture (--set
+# full, 1 launch) of the 128K workload (batch 1, 16q/2kv heads, D=256, page
+# 64, 131,072 + 4 tokens; about 3 GB on the device): dram__bytes_read.sum and
+# dram__bytes_write.sum, and the K/V tokens that launch read.  Reads grow in
+# proportion to the tokens read (every K/V byte crosses HBM once); the writes
+# are the split partials, the same size at any context with the same split
+# count (74 per KV head for batch 1).  So a launch reading `tokens` tokens is
+# credited read_bytes * tokens / captured_tokens + write_bytes.  The figure is
+# reported only while the kernel's code (its sources with comments and
+# whitespace removed) hashes to the value it was captured on; otherwise
+# roofline.traffic is null.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": None,
-    "captured_on": None,
-    "tokens": None,   # K/V tokens read by the captured launch (per sequence, summed)
-    "bytes": None,
+    "sha256": "4a3271ab7a0e9d99da643ebc70ab00386065aa1c636829f7fce37c1c971d3ccd",
+    "captured_on": "128k: verify_tc_kernel<3, 3, 64>, 148 CTAs x 256 threads",
+    "tokens": 131076,
+    "read_bytes": 268745728,
+    "write_bytes": 6563328,
 }
 
 
@@ -603,9 +607,9 @@ def verify_traffic(tokens: int):
     """Captured DRAM bytes of one verify launch, scaled to a launch reading
     `tokens` K/V tokens; None if nothing was captured for this kernel code."""
     t = VERIFY_TRAFFIC
-    if t["bytes"] is None or not t["tokens"] or kernel_code_hash() != t["sha256"]:
+    if t["read_bytes"] is None or not t["tokens"] or kernel_code_hash() != t["sha256"]:
         return None
-    return t["bytes"] * tokens / t["tokens"]
+    return t["read_bytes"] * tokens / t["tokens"] + t["write_bytes"]
 
 
 def workload_desc(args) -> str:

@@ -18,10 +18,12 @@
  *   host during the call and may be freed when it returns.  The library never
  *   allocates device memory.
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
- *   default stream) and never synchronise the host.  The attention kernels
- *   are launched as programmatic dependents of the work before them on the
- *   stream: their set-up may overlap its tail, but they read no global memory
- *   before it has completed, so stream order holds for every input.  The calls
+ *   default stream) and never synchronise the host.  The kernels of the
+ *   attention calls, wmtp_ring_append and wmtp_paged_write are launched as
+ *   programmatic dependents of the work before them on the stream: their
+ *   launch and set-up may overlap its tail, but they touch no global memory
+ *   before it has completed, so stream order holds for every input and
+ *   output.  The calls
  *   can be captured in CUDA graphs (the first call on a device must come
  *   before any capture: it sets kernel attributes).
  * - Host-detectable argument errors return a negative wmtp_status before

@@ -7,9 +7,10 @@
 // are all empty yields o = 0, lse = -inf.
 //
 // Layout of the work: CTA = (row, 128-column block).  Each of the 8 warps
-// takes every 8th split; a lane owns 4 consecutive columns (one float4 per
-// split), so a warp reads 512 contiguous bytes per split and the 8 warps keep
-// many independent loads in flight.  Warp partial sums meet in shared memory.
+// takes every 8th split, up to 8 of them per round with all their loads in
+// flight at once; a lane owns 4 consecutive columns (one float4 per split),
+// so a warp reads 512 contiguous bytes per split.  Warp partial sums meet in
+// shared memory.
 //
 // The kernel is launched as a programmatic dependent of the decode kernel:
 // it may start while the decode kernel drains and waits (griddepcontrol.wait)
@@ -24,6 +25,7 @@ namespace wmtp {
 constexpr int kCombineWarps = 8;
 constexpr int kCombineThreads = 32 * kCombineWarps;
 constexpr int kCombineCols = 128;  // columns per CTA (32 lanes x float4)
+constexpr int kCombineBatch = 8;   // splits whose loads a warp issues together
 
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -54,34 +56,27 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (m != -INFINITY) {
     const float* po = part_o + static_cast<size_t>(row) * nsplit * D + col;
     const bool active = col < D;
-    int s = warp;
-    // two splits per iteration keep two independent loads in flight per lane
-    for (; s + kCombineWarps < nsplit; s += 2 * kCombineWarps) {
-      const float l0 = pl[s];
-      const float l1 = pl[s + kCombineWarps];
-      float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-      if (active) {
-        v0 = *reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D);
-        v1 = *reinterpret_cast<const float4*>(po + static_cast<size_t>(s + kCombineWarps) * D);
+    // warp w takes splits w, w + 8, ...; up to kCombineBatch of them per
+    // round, every load issued before the first is used, so a row costs a
+    // couple of memory round trips instead of one per pair of splits
+    for (int s0 = warp; s0 < nsplit; s0 += kCombineWarps * kCombineBatch) {
+      float4 v[kCombineBatch];
+      float l[kCombineBatch];
+#pragma unroll
+      for (int i = 0; i < kCombineBatch; ++i) {
+        const int s = s0 + i * kCombineWarps;
+        l[i] = s < nsplit ? pl[s] : -INFINITY;
+        v[i] = (s < nsplit && active) ? *reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      const float w0 = (l0 == -INFINITY) ? 0.f : expf(l0 - m);
-      const float w1 = (l1 == -INFINITY) ? 0.f : expf(l1 - m);
-      den += w0 + w1;
-      acc.x += w0 * v0.x + w1 * v1.x;
-      acc.y += w0 * v0.y + w1 * v1.y;
-      acc.z += w0 * v0.z + w1 * v1.z;
-      acc.w += w0 * v0.w + w1 * v1.w;
-    }
-    if (s < nsplit) {
-      const float l0 = pl[s];
-      const float w0 = (l0 == -INFINITY) ? 0.f : expf(l0 - m);
-      den += w0;
-      if (active) {
-        const float4 v0 = *reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D);
-        acc.x += w0 * v0.x;
-        acc.y += w0 * v0.y;
-        acc.z += w0 * v0.z;
-        acc.w += w0 * v0.w;
+#pragma unroll
+      for (int i = 0; i < kCombineBatch; ++i) {
+        const float w = (l[i] == -INFINITY) ? 0.f : expf(l[i] - m);
+        den += w;
+        acc.x += w * v[i].x;
+        acc.y += w * v[i].y;
+        acc.z += w * v[i].z;
+        acc.w += w * v[i].w;
       }
     }
   }

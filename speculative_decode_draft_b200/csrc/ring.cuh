@@ -51,6 +51,11 @@ __global__ void __launch_bounds__(kRingThreads)
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   __shared__ int s_ok, s_len, s_com, s_target, s_n;
+  // launched as a programmatic dependent: wait (unconditionally, before any
+  // memory access) for the work before it on the stream, then let the
+  // attention kernel behind it get scheduled
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     const int len = r.len[b];
     const int com = r.committed[b];
@@ -185,6 +190,11 @@ __global__ void paged_write_kernel(uint4* __restrict__ k_pool, uint4* __restrict
                                    int32_t* status) {
   const int j = blockIdx.x;
   const int b = blockIdx.y;
+  // launched as a programmatic dependent: wait (unconditionally, before any
+  // memory access) for the work before it on the stream, then let the
+  // attention kernel behind it get scheduled
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int p = pos0[b] + j;
   if (p < 0 || p >= max_pages * P) {
     if (threadIdx.x == 0) set_status(status, kDevLenOob);

@@ -80,19 +80,25 @@ wmtp_status ensure_smem_attr(SmemAttrOnce& once, Kern kern, int bytes) {
   return WMTP_OK;
 }
 
-// A launch without attributes whose success is read from the launch call
-// itself, never from cudaGetLastError (which would also report an unrelated
-// earlier error left on this thread, after the kernel had been queued).
+// A launch whose success is read from the launch call itself, never from
+// cudaGetLastError (which would also report an unrelated earlier error left
+// on this thread, after the kernel had been queued).  `programmatic`: launch
+// as a programmatic dependent of the previous work on the stream (the kernel
+// must execute griddepcontrol.wait before its first memory access).
 template <typename... Exp, typename... Act>
-wmtp_status launch_plain(void (*kern)(Exp...), dim3 grid, dim3 block, cudaStream_t st, Act&&... args) {
+wmtp_status launch_plain(bool programmatic, void (*kern)(Exp...), dim3 grid, dim3 block, cudaStream_t st,
+                         Act&&... args) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = programmatic ? attr : nullptr;
+  cfg.numAttrs = programmatic ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...) == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
 }
 
@@ -537,7 +543,7 @@ wmtp_status wmtp_ring_append(const wmtp_params* params, const wmtp_ring* ring, c
   if (speculative && params->gamma_max == 0 && max_new > 0) return WMTP_ERR_INVALID_ARG;
   if (ring->batch == 0) return WMTP_OK;
   RingArgs a = ring_args(params, ring);
-  return launch_plain(ring_append_kernel, dim3(ring->batch), dim3(kRingThreads), static_cast<cudaStream_t>(stream),
+  return launch_plain(true, ring_append_kernel, dim3(ring->batch), dim3(kRingThreads), static_cast<cudaStream_t>(stream),
                       a, truncate_to, n_new, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
                       max_new, speculative ? 1 : 0, status_word);
 }
@@ -547,7 +553,7 @@ wmtp_status wmtp_ring_reset(const wmtp_params* params, const wmtp_ring* ring, vo
   if (s != WMTP_OK) return s;
   if (ring->batch == 0) return WMTP_OK;
   RingArgs a = ring_args(params, ring);
-  return launch_plain(ring_reset_kernel, dim3(256), dim3(256), static_cast<cudaStream_t>(stream), a);
+  return launch_plain(false, ring_reset_kernel, dim3(256), dim3(256), static_cast<cudaStream_t>(stream), a);
 }
 
 wmtp_status wmtp_splitkv_combine(int32_t rows, int32_t head_dim, int32_t nsplit, const float* part_o,
@@ -574,7 +580,7 @@ wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmt
     return WMTP_ERR_INVALID_ARG;
   if (!aligned(kv->k_pool, 16) || !aligned(kv->v_pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
     return WMTP_ERR_INVALID_ARG;
-  return launch_plain(paged_write_kernel, dim3(n_new, batch), dim3(128), static_cast<cudaStream_t>(stream),
+  return launch_plain(true, paged_write_kernel, dim3(n_new, batch), dim3(128), static_cast<cudaStream_t>(stream),
                       static_cast<uint4*>(kv->k_pool), static_cast<uint4*>(kv->v_pool), kv->num_pages,
                       kv->page_table, kv->max_pages, params->page_size, params->num_heads_kv, params->head_dim,
                       pos0, n_new, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),

@@ -43,12 +43,20 @@ def test_workload_strings():
     assert "ctx 65536" in bench.workload_desc(bench.parse(["--ctx", "65536"]))
 
 
+def test_recorded_traffic_matches_the_current_kernel():
+    # the committed capture belongs to the committed kernel code
+    assert bench.kernel_code_hash() == bench.VERIFY_TRAFFIC["sha256"]
+    t = bench.verify_traffic(1048580)
+    assert t is not None and 1.0 < t / (1048580 * 2048) < 1.02
+
+
 def test_traffic_guard_follows_the_kernel_code(tmp_path, monkeypatch):
     # a figure recorded against the current sources, 100 bytes per token
     monkeypatch.setitem(bench.VERIFY_TRAFFIC, "sha256", bench.kernel_code_hash())
     monkeypatch.setitem(bench.VERIFY_TRAFFIC, "tokens", 1000)
-    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "bytes", 100000)
-    assert bench.verify_traffic(4000) == pytest.approx(400000)  # scaled by tokens
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "read_bytes", 100000)
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "write_bytes", 500)
+    assert bench.verify_traffic(4000) == pytest.approx(400500)  # reads scaled by tokens, writes as captured
     # a copy of the sources: a comment edit keeps the figure, a code edit drops it
     for rel in bench.VERIFY_TRAFFIC["sources"]:
         os.makedirs(tmp_path / os.path.dirname(rel), exist_ok=True)
@@ -57,10 +65,10 @@ def test_traffic_guard_follows_the_kernel_code(tmp_path, monkeypatch):
     src = tmp_path / bench.VERIFY_TRAFFIC["sources"][0]
     text = src.read_text()
     src.write_text("// a new comment\n" + text)
-    assert bench.verify_traffic(4000) == pytest.approx(400000)
+    assert bench.verify_traffic(4000) == pytest.approx(400500)
     src.write_text(text.replace("kRescaleLog2 = 8.f", "kRescaleLog2 = 7.f"))
     assert bench.verify_traffic(4000) is None
-    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "bytes", None)
+    monkeypatch.setitem(bench.VERIFY_TRAFFIC, "read_bytes", None)
     assert bench.verify_traffic(4000) is None
 
 
