@@ -582,11 +582,11 @@ def cores_used():
 # roofline.traffic is null.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "4a3271ab7a0e9d99da643ebc70ab00386065aa1c636829f7fce37c1c971d3ccd",
-    "captured_on": "128k: verify_tc_kernel<3, 3, 64>, 148 CTAs x 256 threads",
+    "sha256": "ac88dcb434a755cd457bd8196f2effd5e5546cb6eb22461c8d6be6d2fed4df18",
+    "captured_on": "128k: verify_tc_kernel<3, 3, 64>, 148 CTAs x 384 threads",
     "tokens": 131076,
-    "read_bytes": 268745728,
-    "write_bytes": 6563328,
+    "read_bytes": 268746496,
+    "write_bytes": 4351488,
 }
 
 

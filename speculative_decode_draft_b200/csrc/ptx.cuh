@@ -219,8 +219,8 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
 // base + t/4 + 8.
 //   16x256b.x8 (64 columns, 32 registers): v[4r + {0,1}] = lane t/4, columns
 //     8r + 2(t%4) + {0,1}; v[4r + {2,3}] = lane t/4 + 8, same columns.
-//   16x128b.x8 (32 columns, 16 registers): v[2r] = lane t/4, column
-//     4r + t%4; v[2r + 1] = lane t/4 + 8, same column.
+//   16x128b (4 columns a repetition, 2 registers): v[2r] = lane t/4,
+//     column 4r + t%4; v[2r + 1] = lane t/4 + 8, same column.
 __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* v) {
   asm volatile(
       "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -246,13 +246,29 @@ __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t* v) {
+// 16x256b.x4: the first four repetitions of the x8 layout (32 columns, 16
+// registers).
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t* v) {
   asm volatile(
-      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Two 16x128b.x4 stores (16 columns, 8 registers each: the first four
+// repetitions of the x8 layout) and one wait for both.
+__device__ __forceinline__ void tmem_st_16x128b_x4_pair(uint32_t taddr0, const uint32_t* v, uint32_t taddr1,
+                                                        const uint32_t* w) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%2, %3, %4, %5, %6, %7, %8, %9};\n\t"
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%1], {%10, %11, %12, %13, %14, %15, %16, %17};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr0),
+      "r"(taddr1), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
       : "memory");
 }
 

@@ -22,11 +22,11 @@
 // longer waits for the PV of the tile just before the previous one.
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
 // 16 (r % 4) + r / 4 for M=64, 32 (r % 4) + r / 4 for M=128), so the rows
-// spread over the four lane quadrants and each softmax warp owns a quarter of
-// them.
+// spread over the four lane quadrants and each pair of softmax warps owns a
+// quarter of them.
 //
-// Roles:
-//   warps 0, 7 stream K (warp 0) and V (warp 7) tiles (64 x 256 bf16 each,
+// Roles (12 warps):
+//   warps 0, 3 stream K (warp 0) and V (warp 3) tiles (64 x 256 bf16 each,
 //              128-byte swizzle) into two shared-memory rings (KS and VS tiles
 //              deep) with TMA, one lane each; a K tile is released as soon as
 //              its S = Q K^T has completed, a V tile after its O += P V.  The
@@ -34,16 +34,21 @@
 //              barrier wait holds up the other's issue;
 //   warp 1     allocates the tensor memory; one lane issues S = Q K^T (M rows,
 //              N=64, K from shared memory, K-major);
-//   warp 6     one lane issues O += P V (M rows, N=256, V read MN-major
+//   warp 2     one lane issues O += P V (M rows, N=256, V read MN-major
 //              straight from the TMA tile, bf16).  A lane issues a small
 //              tcgen05.mma only every ~66 cycles, so the two streams issue
 //              from two lanes;
-//   warps 2-5  stage Q into TMEM, then run the softmax.  Each warp covers the
-//              rows of its lane quadrant with sixteen-lane TMEM accesses: four
-//              threads share a row and take 16 of the tile's 64 scores each,
-//              so every lane of the warp works even when a quadrant holds only
-//              8 rows (gamma = 3, G = 8).  Row maxima meet through two
-//              shuffles; P goes back into TMEM.
+//   warps 4-11 stage Q, then run the softmax: two warps per TMEM lane
+//              quadrant (warp % 4), one per half of the tile's 64 columns
+//              (and of O's 256).  A warp covers the rows of its quadrant with
+//              sixteen-lane TMEM accesses: four threads share a row and take
+//              8 of its half's 32 scores each, so every lane works even when
+//              a quadrant holds only 8 rows (gamma = 3, G = 8).  Row maxima
+//              meet through two shuffles, then between the two halves
+//              through shared memory and a two-warp mbarrier; both halves
+//              then take the same rescale decisions.  P goes back into TMEM.
+//              The softmax is the per-tile critical path once a quadrant
+//              holds more than 8 rows (gamma >= 5), so it gets eight warps.
 // The value product is bf16 x bf16 -> fp32 on two MMAs per 16 tokens: P is
 // split into P_hi = bf16(p) and P_lo = bf16(p - P_hi), |p - P_hi - P_lo| <=
 // 2^-16 p (a single bf16 P, 2^-8, would miss a 1e-3 relative-L2 bound), and V
@@ -77,9 +82,11 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 256;       // K producer, QK issuer, 4 softmax warps, PV issuer, V producer
-constexpr int kPvWarp = 6;
-constexpr int kVWarp = 7;
+constexpr int kTcThreads = 384;       // K producer, QK issuer, PV issuer, V producer, 8 softmax warps
+constexpr int kPvWarp = 2;
+constexpr int kVWarp = 3;
+constexpr int kSmWarp0 = 4;           // softmax warps 4..11
+constexpr int kSmThreads = 256;
 constexpr int kBarTmem = 3;           // named barrier: QK issuer + softmax warps
 constexpr int kBarSoftmax = 4;        // named barrier: the softmax warps
 constexpr uint32_t kTmemCols = 512;
@@ -95,13 +102,19 @@ struct TcPlan {
   static constexpr int kOffK = 0;                         // K ring: KS tiles
   static constexpr int kOffV = KS * kTileBytes;           // V ring: VS tiles
   static constexpr int kOffQ = (KS + VS) * kTileBytes;    // Q (QS only), 64 rows, K-major, 128-byte swizzle
+  static constexpr int kH = QS ? 1 : 2;                  // sixteen-lane groups of a quadrant (M / 64)
   static constexpr int kOffBar = kOffQ + (QS ? kTileBytes : 0);
   // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NB], p_full[NB],
-  // pv_done[NB], mma_final, q_ready
-  static constexpr int kNumBars = 2 * KS + 2 * VS + 3 * kNB + 2;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort, split page validity
+  // pv_done[NB], mma_final, q_ready, pair[4 quadrants][2 parities]
+  static constexpr int kNumBars = 2 * KS + 2 * VS + 3 * kNB + 2 + 8;
+  // values the two softmax warps of a quadrant exchange (row maxima, row
+  // sums): [parity][half][quadrant][kH][sub-row][8 row groups] floats
+  static constexpr int kOffXch = kOffBar + kNumBars * 8;
+  static constexpr int kXchBytes = 2 * 2 * 4 * kH * 2 * 8 * 4;
+  static constexpr int kOffMisc = kOffXch + kXchBytes;     // tmem base, abort, split page validity
   static constexpr int kBytes = kOffMisc + 12;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "dynamic shared memory above the 227 KB a CTA may have");
 };
 
 // Depths of the K and V rings (64-token tiles).
@@ -139,7 +152,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kColS = QS ? 0 : 128;  // first score buffer
   constexpr int D = 256;
   static_assert(M == 64 || M == 128, "MMA rows: 64 or 128");
-  constexpr int H = M / 64;  // sixteen-lane halves of a quadrant that hold rows
+  constexpr int H = Plan::kH;  // sixteen-lane groups of a quadrant that hold rows
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -155,6 +168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_pv_done = bar_p_full + 8 * NB;   // [NB]: PV of the tiles using S/P buffer b
   const uint32_t bar_final = bar_pv_done + 8 * NB;
   const uint32_t bar_q_ready = bar_final + 8;
+  const uint32_t bar_pair = bar_q_ready + 8;          // [quadrant][parity]
   volatile int* split_bad = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Plan::kOffMisc + 4);
@@ -182,11 +196,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < NB; ++i) {
       ptx::mbar_init(bar_s_full + 8 * i, 1);
-      ptx::mbar_init(bar_p_full + 8 * i, 4);
+      ptx::mbar_init(bar_p_full + 8 * i, kSmThreads / 32);
       ptx::mbar_init(bar_pv_done + 8 * i, 1);
     }
     ptx::mbar_init(bar_final, 2);  // one commit from each MMA-issuing lane
-    ptx::mbar_init(bar_q_ready, 4);
+    ptx::mbar_init(bar_q_ready, kSmThreads / 32);
+    for (int i = 0; i < 8; ++i) ptx::mbar_init(bar_pair + 8 * i, 2);  // the two warps of a quadrant
     *abort_flag = 0;
     *split_bad = 0;
     ptx::fence_mbar_init();
@@ -199,19 +214,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // the set-up above overlaps the previous kernel's tail
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // ---- Q first: the softmax warps' loads leave before any K/V load of the
-  // CTA.  Thread `lane` of softmax warp q holds row 4 lane + q (zeros for
-  // padding rows); every load is issued before the first use.
-  const int q = warp & 3;  // the TMEM lane quadrant of a softmax warp
-  const bool softmax_warp = warp >= 2 && warp < 6;
-  uint4 qv[D / 8];
+  // CTA.  Thread `lane` of softmax warp (q, half) holds head dims
+  // 128 half .. 128 half + 127 of row 4 lane + q (zeros for padding rows);
+  // every load is issued before the first use.
+  const int q = warp & 3;                   // the TMEM lane quadrant of a softmax warp
+  const int half = (warp - kSmWarp0) >> 2;  // its column half
+  const bool softmax_warp = warp >= kSmWarp0;
+  uint4 qv[D / 16];
   if (softmax_warp) {
     const int row = 4 * lane + q;
     const bool q_active = lane < M / 4 && row < a.rows;
     const __nv_bfloat16* src =
-        q_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D
+        q_active ? a.q + ((static_cast<size_t>(b) * a.num_q + row / a.G) * a.Hq + kvh * a.G + row % a.G) * D +
+                       (D / 2) * half
                  : nullptr;
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j)
+    for (int j = 0; j < D / 16; ++j)
       qv[j] = q_active ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0, 0, 0, 0);
   }
   // the page-table entries of this split's first tiles, guessed from the
@@ -309,10 +327,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (softmax_warp && lane < 16) {
       const int m = 16 * q + lane;
 #pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
+      for (int jj = 0; jj < D / 16; ++jj) {
+        const int j = (D / 16) * half + jj;  // 16-byte unit of the row
         const uint32_t dst = sbase + Plan::kOffQ + (j >> 3) * Plan::kChunkBytes + m * 128 + (((j & 7) ^ (m & 7)) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(qv[j].x), "r"(qv[j].y),
-                     "r"(qv[j].z), "r"(qv[j].w)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(qv[jj].x), "r"(qv[jj].y),
+                     "r"(qv[jj].z), "r"(qv[jj].w)
                      : "memory");
       }
     }
@@ -444,22 +463,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ================================================================= softmax
+    // Warps (q, 0) and (q, 1) share the rows of lane quadrant q; half `half`
+    // takes tile columns 32 half .. 32 half + 31 and O columns
+    // 128 half .. 128 half + 127.
     const uint32_t qlane = static_cast<uint32_t>(32 * q) << 16;
     {
-      // Q of M = 128 goes into TMEM lane 32 q + lane, columns 0..127 (bf16
-      // pairs); Q of M = 64 is already in shared memory
+      // Q of M = 128 goes into TMEM lane 32 q + lane, columns
+      // 64 half .. 64 half + 63 (bf16 pairs of this half's head dims); Q of
+      // M = 64 is already in shared memory
       if constexpr (!QS) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t wq[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            wq[4 * j] = qv[8 * c + j].x;
-            wq[4 * j + 1] = qv[8 * c + j].y;
-            wq[4 * j + 2] = qv[8 * c + j].z;
-            wq[4 * j + 3] = qv[8 * c + j].w;
+            wq[4 * j] = qv[8 * cc + j].x;
+            wq[4 * j + 1] = qv[8 * cc + j].y;
+            wq[4 * j + 2] = qv[8 * cc + j].z;
+            wq[4 * j + 3] = qv[8 * cc + j].w;
           }
-          tc::tmem_st32(tmem_base + qlane + kColQ + 32 * c, wq);
+          tc::tmem_st32(tmem_base + qlane + kColQ + 64 * half + 32 * cc, wq);
         }
         tc::fence_before_sync();
       }
@@ -467,14 +490,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) ptx::mbar_arrive(bar_q_ready);
     }
 
-    // Sixteen-lane view: in half h this thread covers TMEM lanes
+    // Sixteen-lane view: in group h this thread covers TMEM lanes
     // 16 h + lane / 4 (sub-row j = 0) and 16 h + lane / 4 + 8 (j = 1) of the
-    // quadrant, and columns 8 r + 2 (lane % 4) + {0, 1} of every 8 (r = 0..7).
-    // The four threads lane / 4 * 4 + {0..3} share both rows.
+    // quadrant, and of this half's 32 columns of a tile columns
+    // 32 half + 8 r + 2 (lane % 4) + {0, 1} (r = 0..3).  The four threads
+    // lane / 4 * 4 + {0..3} share both rows.
     const int cq = 2 * (lane & 3);
     int row_of[H][2];
     bool act[H][2];    // this thread's row exists
-    bool any_r[H][2];  // some row of this warp's (half, sub-row) group exists (warp-uniform)
+    bool any_r[H][2];  // some row of this warp's (group, sub-row) exists (warp-uniform)
     int lim[H][2];     // causal limit (exclusive)
     const int q_first = a.q_pos0 != nullptr ? a.q_pos0[b] : n_tok - a.num_q;
 #pragma unroll
@@ -496,7 +520,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         m_ref[h][j] = -INFINITY;
-        l_run[h][j] = 0.f;  // this thread's share (16 of the 64 columns of every tile)
+        l_run[h][j] = 0.f;  // this thread's share (8 of this half's 32 columns of every tile)
         m_g[h][j] = -INFINITY;
         have_g[h][j] = false;
       }
@@ -508,8 +532,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const size_t grow = (static_cast<size_t>(b) * a.num_q + r / a.G) * a.Hq + kvh * a.G + r % a.G;
       return a.part_o + (grow * a.nsplit + split) * D;
     };
+    // O columns 64 cb .. 64 cb + 63 of group h; this half owns cb = 2 half, 2 half + 1
     auto o_addr = [&](int h, int cb) -> uint32_t {
       return tmem_base + qlane + (static_cast<uint32_t>(16 * h) << 16) + kColO + 64 * cb;
+    };
+    auto s_addr_of = [&](int h, int sb) -> uint32_t {
+      return tmem_base + qlane + (static_cast<uint32_t>(16 * h) << 16) + kColS + sb * 64;
+    };
+    // Exchange with the other half of the quadrant.  Step s (tile s, or
+    // my_tiles for the row sums at the end) writes slots of parity s & 1 and
+    // completes a phase of pair barrier (q, s & 1); a warp reaches step s + 2
+    // only after its partner has arrived at step s + 1, so by then the
+    // partner has read the slots of step s.
+    float* xch = reinterpret_cast<float*>(smem + Plan::kOffXch);
+    auto xslot = [&](int s, int hf, int h, int j) -> float* {
+      return xch + (((((s & 1) * 2 + hf) * 4 + q) * H + h) * 2 + j) * 8 + (lane >> 2);
+    };
+    auto pair_sync = [&](int s) -> bool {
+      const uint32_t bar = bar_pair + 8 * (2 * q + (s & 1));
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar);
+      const bool ok = __all_sync(0xffffffffu, tc_wait(bar, (s >> 1) & 1, abort_flag));
+      tc::fence_after_sync();
+      return ok;
     };
 
     // Page validity, once for the whole split: a tile with a page outside the
@@ -520,12 +566,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int box_rows = min(a.page_size, kTileTokens);
       const int first = t_begin * kTileTokens, last = min(t_end * kTileTokens, n_tok);
       bool ok = true;
-      for (int tok = first + (threadIdx.x - 64) * box_rows; tok < last; tok += 128 * box_rows) {
+      for (int tok = first + (threadIdx.x - kSmWarp0 * 32) * box_rows; tok < last; tok += kSmThreads * box_rows) {
         const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + tok / a.page_size];
         ok = ok && pg >= 0 && pg < a.num_pages;
       }
       if (!__all_sync(0xffffffffu, ok) && lane == 0) *split_bad = 1;
-      ptx::named_bar_sync(kBarSoftmax, 128);
+      ptx::named_bar_sync(kBarSoftmax, kSmThreads);
     }
     const bool split_ok = *split_bad == 0;
 
@@ -547,7 +593,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the current reference: G = G 2^(m_g - m_ref) + O; PV(k) then starts
         // a fresh accumulation.  PV(k-1) completes the pv_done phase of its
         // buffer; the buffer's next phase needs P(k-1+NB), so the wait is
-        // unambiguous.
+        // unambiguous.  Each half folds its own O columns.
         if (!__all_sync(0xffffffffu, tc_wait(bar_pv_done + 8 * ((k - 1) % NB), ((k - 1) / NB) & 1, abort_flag))) {
           failed = true;
           break;
@@ -561,7 +607,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int j = 0; j < 2; ++j) gs[j] = have_g[h][j] ? ptx::ex2(m_g[h][j] - m_ref[h][j]) : 0.f;
 #pragma unroll 1
-          for (int cb = 0; cb < 4; ++cb) {
+          for (int cb = 2 * half; cb < 2 * half + 2; ++cb) {
             uint32_t o[32];
             tc::tmem_ld_16x256b_x8(o_addr(h, cb), o);
 #pragma unroll
@@ -605,7 +651,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t vt = sbase + Plan::kOffV + stage * Plan::kTileBytes;
         // 16-byte unit c (0..31) of token row r: chunk c / 8, unit c % 8 (a
         // whole row is zeroed, so the swizzle does not matter)
-        for (int u = threadIdx.x - 64; u < (kTileTokens - r0) * 32; u += 128) {
+        for (int u = threadIdx.x - kSmWarp0 * 32; u < (kTileTokens - r0) * 32; u += kSmThreads) {
           const int r = r0 + u / 32, c = u % 32;
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vt + (c >> 3) * Plan::kChunkBytes +
                                                                        r * 128 + ((c & 7) << 4)),
@@ -615,60 +661,84 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::fence_proxy_async_smem();
       }
 
+      // this half's scores, scaled to log2 units (masked entries -inf), and
+      // their row maxima
+      float x[H][2][8];
+      float mx[H][2];
 #pragma unroll
       for (int h = 0; h < H; ++h) {
-        const uint32_t s_addr = tmem_base + qlane + (static_cast<uint32_t>(16 * h) << 16) + kColS + sb * 64;
-        uint32_t ph[16], pl[16];
+        mx[h][0] = mx[h][1] = -INFINITY;
+        if (!(any_r[h][0] || any_r[h][1])) continue;
+        uint32_t sraw[16];
+        tc::tmem_ld_16x256b_x4(s_addr_of(h, sb) + 32 * half, sraw);
+        // sub-row groups without any row are skipped (warp-uniform); a tile
+        // without masked positions takes the short path
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ph[i] = pl[i] = 0u;
-        if (any_r[h][0] || any_r[h][1]) {
-          uint32_t sraw[32];
-          tc::tmem_ld_16x256b_x8(s_addr, sraw);
-          float x[2][16];
-          float mx[2] = {-INFINITY, -INFINITY};
-          // sub-row groups without any row are skipped (warp-uniform); a
-          // tile without masked positions takes the short path
+        for (int j = 0; j < 2; ++j) {
+          if (!any_r[h][j]) continue;
+          if (!masked_tile) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            if (!any_r[h][j]) continue;
-            if (!masked_tile) {
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-              for (int r = 0; r < 8; ++r)
+              for (int e = 0; e < 2; ++e)
+                x[h][j][2 * r + e] = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
+          } else {
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
-                  x[j][2 * r + e] = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
-            } else {
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-              for (int r = 0; r < 8; ++r)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  const int t = tok0 + 8 * r + cq + e;
-                  const float s = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
-                  x[j][2 * r + e] = (tile_ok && t < lim[h][j] && t < n_tok) ? s : -INFINITY;
-                }
-            }
-            // pairwise maximum (a tree keeps the dependent chain short)
-            float t8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) t8[i] = fmaxf(x[j][2 * i], x[j][2 * i + 1]);
-#pragma unroll
-            for (int w2 = 4; w2 > 0; w2 >>= 1)
-#pragma unroll
-              for (int i = 0; i < w2; ++i) t8[i] = fmaxf(t8[i], t8[i + w2]);
-            mx[j] = t8[0];
-            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 1));
-            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 2));
+              for (int e = 0; e < 2; ++e) {
+                const int t = tok0 + 32 * half + 8 * r + cq + e;
+                const float s = __uint_as_float(sraw[4 * r + 2 * j + e]) * a.scale_log2;
+                x[h][j][2 * r + e] = (tile_ok && t < lim[h][j] && t < n_tok) ? s : -INFINITY;
+              }
           }
+          // pairwise maximum (a tree keeps the dependent chain short)
+          float t4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) t4[i] = fmaxf(x[h][j][2 * i], x[h][j][2 * i + 1]);
+          float m = fmaxf(fmaxf(t4[0], t4[2]), fmaxf(t4[1], t4[3]));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+          mx[h][j] = m;
+        }
+      }
+      // the other half's maxima (both halves then hold the tile maximum of
+      // every row and take the same decisions below).  The S columns this
+      // warp reads are the P columns its partner writes: both loads complete
+      // before the exchange, both stores come after it.
+      if ((lane & 3) == 0) {
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (any_r[h][j]) *xslot(k, half, h, j) = mx[h][j];
+      }
+      if (!pair_sync(k)) {
+        failed = true;
+        break;
+      }
+#pragma unroll
+      for (int h = 0; h < H; ++h)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          if (any_r[h][j]) mx[h][j] = fmaxf(mx[h][j], *xslot(k, half ^ 1, h, j));
+
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        uint32_t ph[8], pl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ph[i] = pl[i] = 0u;
+        if (any_r[h][0] || any_r[h][1]) {
           // raise the reference maximum only when the tile exceeds it by more
           // than 2^8; rows whose reference moved rescale their O row and sum
           float alpha[2] = {1.f, 1.f};
           bool moved = false;
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            if (mx[j] > m_ref[h][j] + kRescaleLog2 || (m_ref[h][j] == -INFINITY && mx[j] != -INFINITY)) {
-              alpha[j] = (m_ref[h][j] == -INFINITY) ? 0.f : ptx::ex2(m_ref[h][j] - mx[j]);
+            if (mx[h][j] > m_ref[h][j] + kRescaleLog2 || (m_ref[h][j] == -INFINITY && mx[h][j] != -INFINITY)) {
+              alpha[j] = (m_ref[h][j] == -INFINITY) ? 0.f : ptx::ex2(m_ref[h][j] - mx[h][j]);
               moved = moved || m_ref[h][j] != -INFINITY;
-              m_ref[h][j] = mx[j];
+              m_ref[h][j] = mx[h][j];
             }
             l_run[h][j] *= alpha[j];
           }
@@ -686,7 +756,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               o_ready = true;
             }
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 2 * half; cb < 2 * half + 2; ++cb) {
               uint32_t o[32];
               tc::tmem_ld_16x256b_x8(o_addr(h, cb), o);
 #pragma unroll
@@ -699,29 +769,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tc::tmem_st_16x256b_x8(o_addr(h, cb), o);
             }
           }
-          // P = 2^(x - m_ref) as bf16 hi + lo pairs (token pair 4 r + lane % 4
-          // of the row), back into the S columns
+          // P = 2^(x - m_ref) as bf16 hi + lo pairs: token pair
+          // 16 half + 4 r + lane % 4 of the tile, back into the S columns
+          // (P_hi in columns 0..31, P_lo in 32..63)
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             if (!any_r[h][j]) continue;
             const float base = (m_ref[h][j] == -INFINITY) ? 0.f : m_ref[h][j];
-            float ps[8];
+            float ps[4];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-              const float p0 = ptx::ex2(x[j][2 * r] - base);  // 2^-inf = 0 for masked entries
-              const float p1 = ptx::ex2(x[j][2 * r + 1] - base);
+            for (int r = 0; r < 4; ++r) {
+              const float p0 = ptx::ex2(x[h][j][2 * r] - base);  // 2^-inf = 0 for masked entries
+              const float p1 = ptx::ex2(x[h][j][2 * r + 1] - base);
               ps[r] = p0 + p1;
               split_pack(p0, p1, ph[2 * r + j], pl[2 * r + j]);
             }
-#pragma unroll
-            for (int w2 = 4; w2 > 0; w2 >>= 1)
-#pragma unroll
-              for (int i = 0; i < w2; ++i) ps[i] += ps[i + w2];
-            l_run[h][j] += ps[0];
+            l_run[h][j] += (ps[0] + ps[2]) + (ps[1] + ps[3]);
           }
         }
-        tc::tmem_st_16x128b_x8(s_addr, ph);
-        tc::tmem_st_16x128b_x8(s_addr + 32, pl);
+        const uint32_t s_addr = s_addr_of(h, sb);
+        tc::tmem_st_16x128b_x4_pair(s_addr + 16 * half, ph, s_addr + 32 + 16 * half, pl);
       }
       if (failed) break;
 
@@ -736,6 +803,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!__all_sync(0xffffffffu, tc_wait(bar_final, 0, abort_flag))) failed = true;
       tc::fence_after_sync();
     }
+    // the row sums: the four threads of a row hold a quarter of this half's
+    // share, the other half's warp the rest
+#pragma unroll
+    for (int h = 0; h < H; ++h)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float l = l_run[h][j];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        l_run[h][j] = l;
+      }
+    if (!failed) {
+      if ((lane & 3) == 0) {
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (any_r[h][j]) *xslot(my_tiles, half, h, j) = l_run[h][j];
+      }
+      if (!pair_sync(my_tiles)) {
+        failed = true;
+      } else {
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (any_r[h][j]) l_run[h][j] += *xslot(my_tiles, half ^ 1, h, j);
+      }
+    }
     failed = __any_sync(0xffffffffu, failed || *abort_flag != 0);
     if (failed) {
       if (lane == 0) set_status(a.status, kDevTimeout);
@@ -746,17 +842,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float inv[2], gs[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        // the row's sum: each of its four threads holds a quarter
-        float l = l_run[h][j];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        l_run[h][j] = l;
-        inv[j] = (l > 0.f && !failed) ? 1.f / l : 0.f;
+        inv[j] = (l_run[h][j] > 0.f && !failed) ? 1.f / l_run[h][j] : 0.f;
         gs[j] = (have_g[h][j] && !failed) ? ptx::ex2(m_g[h][j] - m_ref[h][j]) : 0.f;
       }
       if (!(any_r[h][0] || any_r[h][1])) continue;
 #pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
+      for (int cb = 2 * half; cb < 2 * half + 2; ++cb) {
         uint32_t o[32];
         if (my_tiles > 0 && !failed) {
           tc::tmem_ld_16x256b_x8(o_addr(h, cb), o);
@@ -779,7 +870,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        if (act[h][j] && (lane & 3) == 0) {
+        if (half == 0 && act[h][j] && (lane & 3) == 0) {
           const int r = row_of[h][j];
           const size_t grow = (static_cast<size_t>(b) * a.num_q + r / a.G) * a.Hq + kvh * a.G + r % a.G;
           // m_ref is in log2 units of the scaled score
@@ -794,7 +885,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ---- every MMA has completed (the MMA lanes waited for their final
   // commit); free the tensor memory
-  ptx::named_bar_sync(kBarTmem, 160);
+  ptx::named_bar_sync(kBarTmem, 32 + kSmThreads);
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem_base, kTmemCols);
