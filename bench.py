@@ -672,24 +672,35 @@ def time_arms(args, wk, world: int, make_clocks=None) -> dict:
     if int(wk.status.item()) != 0:
         raise SystemExit(f"device status {int(wk.status.item()):#x} during warmup")
 
-    # One CUDA graph per timed decode step and arm (the step's ~40 library
-    # launches replay without host gaps); --eager launches them from Python.
-    graphs = {}
+    # Two CUDA graphs per timed decode step and arm (the step's ~40 library
+    # launches replay without host gaps): the plain step, which the step
+    # times come from, and the same step with an event pair around every
+    # attention call, for the per-call means.  An event node between two
+    # kernels ends the programmatic overlap of the second with the first, so
+    # the instrumented step runs slower than the plain one.  --eager launches
+    # the steps from Python instead.
+    graphs, graphs_ev = {}, {}
     if not args.eager:
         for arm in ("windowed", "native"):
-            graphs[arm] = []
+            graphs[arm], graphs_ev[arm] = [], []
             for s in range(args.warmup, args.warmup + args.steps):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    wk.step(s, arm)
+                graphs[arm].append(g)
                 evs = []
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
                     wk.step(s, arm, ev=evs, external_events=True)
-                graphs[arm].append((g, evs))
+                graphs_ev[arm].append((g, evs))
         torch.cuda.synchronize()
 
-    def timed_interleaved():
+    def timed_interleaved(instrumented: bool):
         """K decode steps of each arm, alternating windowed and native step by
         step so both arms see the same clocks and power state; each step is
-        bracketed by its own events and an arm's time is the sum of its steps."""
+        bracketed by its own events and an arm's time is the sum of its steps.
+        `instrumented`: replay the steps with per-call events (their
+        per-call spans are returned; their step times are not used)."""
         evs = {"windowed": [], "native": []}
         spans = {"windowed": [], "native": []}
         wk.restore_ring(ring_after_warmup)
@@ -700,12 +711,14 @@ def time_arms(args, wk, world: int, make_clocks=None) -> dict:
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record()
-                if graphs:
-                    g, gev = graphs[arm][i]
+                if graphs and instrumented:
+                    g, gev = graphs_ev[arm][i]
                     g.replay()
                     evs[arm].extend(gev)
+                elif graphs:
+                    graphs[arm][i].replay()
                 else:
-                    wk.step(s, arm, ev=evs[arm])
+                    wk.step(s, arm, ev=evs[arm] if instrumented else None)
                 b.record()
                 spans[arm].append((a, b))
         torch.cuda.synchronize()
@@ -716,8 +729,9 @@ def time_arms(args, wk, world: int, make_clocks=None) -> dict:
     # the windowed arm advances the ring; the native arm must not see a
     # different ring, and neither reads the other's state
     clocks = make_clocks() if make_clocks else None
-    ms_arm, ev_arm = timed_interleaved()
+    ms_arm, _ = timed_interleaved(False)
     clk = clocks.stop() if clocks else None
+    _, ev_arm = timed_interleaved(True)
     ms_win = max_over_ranks(ms_arm["windowed"], world)
     ms_nat = max_over_ranks(ms_arm["native"], world)
     ev_win, ev_nat = ev_arm["windowed"], ev_arm["native"]
@@ -764,33 +778,45 @@ def run_sweep(args, rank: int, world: int, dev) -> int:
 
 def time_single_arm(args, wk, arm: str, world: int) -> dict:
     """Warm up one arm, capture each timed step as a CUDA graph, time K steps
-    between a barrier + synchronize on both sides (max over ranks)."""
+    between a barrier + synchronize on both sides (max over ranks); then
+    replay the same steps with an event pair around every attention call for
+    the per-call means (as in time_arms, the step time comes from the plain
+    graphs)."""
     import torch
     for s in range(args.warmup):
         wk.step(s, arm)
     torch.cuda.synchronize()
-    graphs = []
+    ring0 = wk.snapshot_ring()
+    graphs, graphs_ev = [], []
     for s in range(args.warmup, args.warmup + args.steps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            wk.step(s, arm)
+        graphs.append(g)
         evs = []
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             wk.step(s, arm, ev=evs, external_events=True)
-        graphs.append((g, evs))
+        graphs_ev.append((g, evs))
     torch.cuda.synchronize()
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for g, _ in graphs:
+    for g in graphs:
         g.replay()
     b.record()
     torch.cuda.synchronize()
     barrier(world)
+    wk.restore_ring(ring0)
+    for g, _ in graphs_ev:
+        g.replay()
+    torch.cuda.synchronize()
     per = {}
-    for _, evs in graphs:
+    for _, evs in graphs_ev:
         for kind, e0, e1 in evs:
             per.setdefault(kind, []).append(e0.elapsed_time(e1) * 1000.0)
     ms = max_over_ranks(a.elapsed_time(b), world)
-    del graphs
+    del graphs, graphs_ev
     return {"us_per_step": ms * 1000.0 / args.steps, "per_call_us": {k: statistics.mean(v) for k, v in per.items()}}
 
 
@@ -1071,7 +1097,8 @@ def main():
                   "between the draft steps of one decode step",
             "launch": "eager Python launches" if args.eager else "one CUDA graph per decode step and arm",
             "timing": "windowed and native steps alternate; each arm's time is the sum of its steps' CUDA-event "
-                      "spans on the launching stream",
+                      "spans on the launching stream; per-call times come from a second pass over the same steps "
+                      "with an event pair around each call",
             "native_us_per_step": us_nat,
             "windowed_us_per_step": us_win,
             "native_over_windowed": us_nat / us_win,

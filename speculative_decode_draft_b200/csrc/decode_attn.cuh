@@ -49,7 +49,7 @@
 // weights and values of one sign that loss is systematic (~n 2^-25 of the
 // result after n tokens).  Every kRunTiles tiles the accumulator is therefore
 // folded into the split's fp32 partial in global memory with exact fp32 adds
-// and restarted, so one accumulation spans at most 8,192 tokens.
+// and restarted, so one accumulation spans at most 16,384 tokens.
 #pragma once
 
 #include <cuda.h>
@@ -67,7 +67,7 @@ constexpr int kThreads = 32 * (kComputeWarps + 1);
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kPPitchBytes = 144;  // one P row: 64 bf16 + 16 bytes of padding
 constexpr int kBarCompute = 1;     // named barrier id of the compute warps
-constexpr int kRunTiles = 128;     // tiles per accumulation run (8,192 tokens)
+constexpr int kRunTiles = 256;     // tiles per accumulation run (16,384 tokens)
 
 // Status bits (mirror include/wmtp.h).
 constexpr int kDevPageOob = 0x1;

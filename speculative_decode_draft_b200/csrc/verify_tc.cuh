@@ -64,7 +64,7 @@
 // loss is systematic, ~n 2^-25 of the result after n products.  Every
 // kRunTiles tiles the softmax threads therefore fold the accumulator into the
 // split's fp32 partial in global memory (exact fp32 adds) and the next PV
-// starts a fresh accumulation; a run then spans at most 8,192 tokens
+// starts a fresh accumulation; a run then spans at most 16,384 tokens
 // (kRunTiles, shared with the mma.sync kernel).
 //
 // Every mbarrier wait is bounded; a wait that gives up raises

@@ -233,7 +233,7 @@ def test_native_draft_flat_sea_in_one_long_split():
     sequence and KV head, so one CTA accumulates a whole million-token
     context.  With nearly equal weights and values of one sign (mean 2) an
     accumulation that drops the low-order bits of each product against the
-    running sum would bias the result by ~0.5%; the kernel's runs of 8,192
+    running sum would bias the result by ~0.5%; the kernel's runs of 16,384
     tokens keep it inside the parity bar."""
     G, Hkv, D, P, B = 8, 2, 256, 64, 64
     Hq = G * Hkv
