@@ -363,13 +363,19 @@ class Workload:
         """One decode step.  ``inputs`` (a dict like ``step_inputs``) replaces
         the resident inputs of step ``s``; ``outputs`` (``{"draft": [gamma,
         ...], "verify": [L, ...]}``, e.g. pinned host buffers) receives every
-        attention output of the step."""
+        attention output of the step.  With ``ev`` one draft call and one
+        verify call of the step (draft s mod gamma, layer s mod L) are
+        bracketed by an event pair: an event node between two kernels ends the
+        second one's programmatic overlap with the first, so the other calls
+        keep theirs."""
         torch, w = self.torch, self.w
 
         def E(**kw):  # events inside a captured graph must be graph nodes
             return torch.cuda.Event(external=external_events, **kw)
         x = inputs if inputs is not None else self.step_inputs(s)
+        ev_all = ev
         for j in range(self.gamma):
+            ev = ev_all if j == s % self.gamma else None
             if arm == "windowed":
                 w.ring_append(self.p, self.ring, x["k_draft"][j], x["v_draft"][j], self.one,
                               speculative=True, status=self.status)
@@ -394,6 +400,7 @@ class Workload:
             if outputs is not None:
                 outputs["draft"][j].copy_(self.o_draft, non_blocking=True)
         for l in range(self.L):
+            ev = ev_all if l == s % self.L else None
             c = self.caches[l]
             c.kv_len = x["len_ver"]
             w.paged_write(self.p, c, x["pos_ver"], x["k_ver"][l], x["v_ver"][l], status=self.status)
@@ -672,35 +679,26 @@ def time_arms(args, wk, world: int, make_clocks=None) -> dict:
     if int(wk.status.item()) != 0:
         raise SystemExit(f"device status {int(wk.status.item()):#x} during warmup")
 
-    # Two CUDA graphs per timed decode step and arm (the step's ~40 library
-    # launches replay without host gaps): the plain step, which the step
-    # times come from, and the same step with an event pair around every
-    # attention call, for the per-call means.  An event node between two
-    # kernels ends the programmatic overlap of the second with the first, so
-    # the instrumented step runs slower than the plain one.  --eager launches
-    # the steps from Python instead.
-    graphs, graphs_ev = {}, {}
+    # One CUDA graph per timed decode step and arm (the step's ~40 library
+    # launches replay without host gaps); --eager launches them from Python.
+    # Each step brackets one draft call and one verify call with events (the
+    # per-call means); the other calls run as the product runs them.
+    graphs = {}
     if not args.eager:
         for arm in ("windowed", "native"):
-            graphs[arm], graphs_ev[arm] = [], []
+            graphs[arm] = []
             for s in range(args.warmup, args.warmup + args.steps):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    wk.step(s, arm)
-                graphs[arm].append(g)
                 evs = []
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
                     wk.step(s, arm, ev=evs, external_events=True)
-                graphs_ev[arm].append((g, evs))
+                graphs[arm].append((g, evs))
         torch.cuda.synchronize()
 
-    def timed_interleaved(instrumented: bool):
+    def timed_interleaved():
         """K decode steps of each arm, alternating windowed and native step by
         step so both arms see the same clocks and power state; each step is
-        bracketed by its own events and an arm's time is the sum of its steps.
-        `instrumented`: replay the steps with per-call events (their
-        per-call spans are returned; their step times are not used)."""
+        bracketed by its own events and an arm's time is the sum of its steps."""
         evs = {"windowed": [], "native": []}
         spans = {"windowed": [], "native": []}
         wk.restore_ring(ring_after_warmup)
@@ -711,14 +709,12 @@ def time_arms(args, wk, world: int, make_clocks=None) -> dict:
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record()
-                if graphs and instrumented:
-                    g, gev = graphs_ev[arm][i]
+                if graphs:
+                    g, gev = graphs[arm][i]
                     g.replay()
                     evs[arm].extend(gev)
-                elif graphs:
-                    graphs[arm][i].replay()
                 else:
-                    wk.step(s, arm, ev=evs[arm] if instrumented else None)
+                    wk.step(s, arm, ev=evs[arm])
                 b.record()
                 spans[arm].append((a, b))
         torch.cuda.synchronize()
@@ -729,9 +725,8 @@ def time_arms(args, wk, world: int, make_clocks=None) -> dict:
     # the windowed arm advances the ring; the native arm must not see a
     # different ring, and neither reads the other's state
     clocks = make_clocks() if make_clocks else None
-    ms_arm, _ = timed_interleaved(False)
+    ms_arm, ev_arm = timed_interleaved()
     clk = clocks.stop() if clocks else None
-    _, ev_arm = timed_interleaved(True)
     ms_win = max_over_ranks(ms_arm["windowed"], world)
     ms_nat = max_over_ranks(ms_arm["native"], world)
     ev_win, ev_nat = ev_arm["windowed"], ev_arm["native"]
@@ -778,45 +773,33 @@ def run_sweep(args, rank: int, world: int, dev) -> int:
 
 def time_single_arm(args, wk, arm: str, world: int) -> dict:
     """Warm up one arm, capture each timed step as a CUDA graph, time K steps
-    between a barrier + synchronize on both sides (max over ranks); then
-    replay the same steps with an event pair around every attention call for
-    the per-call means (as in time_arms, the step time comes from the plain
-    graphs)."""
+    between a barrier + synchronize on both sides (max over ranks)."""
     import torch
     for s in range(args.warmup):
         wk.step(s, arm)
     torch.cuda.synchronize()
-    ring0 = wk.snapshot_ring()
-    graphs, graphs_ev = [], []
+    graphs = []
     for s in range(args.warmup, args.warmup + args.steps):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            wk.step(s, arm)
-        graphs.append(g)
         evs = []
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             wk.step(s, arm, ev=evs, external_events=True)
-        graphs_ev.append((g, evs))
+        graphs.append((g, evs))
     torch.cuda.synchronize()
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for g in graphs:
+    for g, _ in graphs:
         g.replay()
     b.record()
     torch.cuda.synchronize()
     barrier(world)
-    wk.restore_ring(ring0)
-    for g, _ in graphs_ev:
-        g.replay()
-    torch.cuda.synchronize()
     per = {}
-    for _, evs in graphs_ev:
+    for _, evs in graphs:
         for kind, e0, e1 in evs:
             per.setdefault(kind, []).append(e0.elapsed_time(e1) * 1000.0)
     ms = max_over_ranks(a.elapsed_time(b), world)
-    del graphs, graphs_ev
+    del graphs
     return {"us_per_step": ms * 1000.0 / args.steps, "per_call_us": {k: statistics.mean(v) for k, v in per.items()}}
 
 
@@ -1097,8 +1080,8 @@ def main():
                   "between the draft steps of one decode step",
             "launch": "eager Python launches" if args.eager else "one CUDA graph per decode step and arm",
             "timing": "windowed and native steps alternate; each arm's time is the sum of its steps' CUDA-event "
-                      "spans on the launching stream; per-call times come from a second pass over the same steps "
-                      "with an event pair around each call",
+                      "spans on the launching stream; per-call times from an event pair around one draft call "
+                      "and one verify call of each timed step (draft s mod gamma, layer s mod L)",
             "native_us_per_step": us_nat,
             "windowed_us_per_step": us_win,
             "native_over_windowed": us_nat / us_win,
