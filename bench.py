@@ -176,11 +176,15 @@ class ClockSampler:
         self.running = False
         self.thread.join(timeout=5)
         nv = self.nv
-        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
-                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
-                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
-                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
-                "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown}
+        # every clock-event reason NVML reports except idle (a leftover clock
+        # lock shows as applications_clocks_setting)
+        names = {"hw_slowdown": "HwSlowdown", "hw_thermal_slowdown": "HwThermalSlowdown",
+                 "sw_thermal_slowdown": "SwThermalSlowdown", "sw_power_cap": "SwPowerCap",
+                 "hw_power_brake_slowdown": "HwPowerBrakeSlowdown",
+                 "applications_clocks_setting": "ApplicationsClocksSetting", "sync_boost": "SyncBoost",
+                 "display_clock_setting": "DisplayClockSetting"}
+        bits = {k: getattr(nv, "nvmlClocksEventReason" + v) for k, v in names.items()
+                if hasattr(nv, "nvmlClocksEventReason" + v)}
         if not self.samples:
             return None
         reasons = sorted({name for _, r in self.samples for name, bit in bits.items() if r & bit})
