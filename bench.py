@@ -1018,12 +1018,18 @@ def main():
         flat = {}
         q1 = wk.q_draft[args.warmup][0][:1].contiguous()
         o1, l1 = wk.o_draft[:1], wk.l_draft[:1]
+        rings = {}
         for c in (32768, 131072, 1048576):
-            ring = w.Ring.allocate(wk.p, 1, dev)
-            fill_ring_to(wk.p, ring, c, seed=c, device=dev)
-            flat[str(c)] = graph_call_us(lambda: w.draft_attn_windowed(
-                wk.p, q1, ring, out=o1, lse=l1, workspace=wk.workspace, status=wk.status))
-            del ring
+            rings[c] = w.Ring.allocate(wk.p, 1, dev)
+            fill_ring_to(wk.p, rings[c], c, seed=c, device=dev)
+        # two interleaved rounds, the better time per context: the first
+        # measurement after the timed region ran slower whichever context it was
+        for _ in range(2):
+            for c, ring in rings.items():
+                t = graph_call_us(lambda: w.draft_attn_windowed(
+                    wk.p, q1, ring, out=o1, lse=l1, workspace=wk.workspace, status=wk.status))
+                flat[str(c)] = min(t, flat.get(str(c), math.inf))
+        del rings
         torch.cuda.empty_cache()
 
     # a read-only streaming reference (torch's sum over 4 GiB; context for the

@@ -38,14 +38,20 @@ def test_windowed_draft_time_is_flat_in_context(window):
     lse = torch.empty(1, 16, dtype=torch.float32, device=DEV)
     ws = torch.empty(w.workspace_bytes("windowed", p, 1), dtype=torch.uint8, device=DEV)
     status = w.new_status(DEV)
-    times = {}
+    rings = {}
     for ctx in (32768, 131072, 1048576):
-        ring = w.Ring.allocate(p, 1, DEV)
-        fill_ring_to(p, ring, ctx, seed=ctx, device=DEV)
-        times[ctx] = graph_call_us(lambda: w.draft_attn_windowed(p, q, ring, out=out, lse=lse, workspace=ws,
-                                                                  status=status))
-        assert int(ring.len.item()) == ctx
-        del ring
+        rings[ctx] = w.Ring.allocate(p, 1, DEV)
+        fill_ring_to(p, rings[ctx], ctx, seed=ctx, device=DEV)
+        assert int(rings[ctx].len.item()) == ctx
+    # two interleaved rounds, the better time per context (the first
+    # measurement of a series can run slower whichever context it is)
+    times = {}
+    for _ in range(2):
+        for ctx, ring in rings.items():
+            t = graph_call_us(lambda: w.draft_attn_windowed(p, q, ring, out=out, lse=lse, workspace=ws,
+                                                             status=status))
+            times[ctx] = min(t, times.get(ctx, float("inf")))
+    del rings
     assert int(status.item()) == 0
     mid = statistics.median(times.values())
     for ctx, t in times.items():
