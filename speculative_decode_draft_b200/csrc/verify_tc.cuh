@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int t_end = min(t_begin + tps, ntiles);
   const int my_tiles = t_end - t_begin;
 
-  // ---- producers: warp 0 loads K tiles, warp 7 V tiles (lane 0 each), each
+  // ---- producers: warp 0 loads K tiles, warp 3 V tiles (lane 0 each), each
   // into its own ring.  Tile k of a ring goes to stage k % depth.
   const bool is_k = warp == 0;
   const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
