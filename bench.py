@@ -1009,6 +1009,25 @@ def main():
         win_paged_us = b0.elapsed_time(b1) * 1000.0 / 10
         del g
 
+    # verify (layer 0) and the native draft, ten calls back to back in one
+    # CUDA graph: each call's launch and ramp overlap the previous call's tail
+    # (programmatic launches), which the bracketed per-call times above cannot
+    # show; context for the roofline, which uses the bracketed verify time
+    b2b = None
+    if not args.sweep:
+        from speculative_decode_draft_b200.timing import graph_call_us
+        s0 = args.warmup
+        c0 = wk.caches[0]
+        c0.kv_len = wk.len_ver[s0]
+        ver_b2b = graph_call_us(lambda: w.verify_attn(wk.p, wk.q_ver[s0][0], c0, out=wk.o_ver, lse=wk.l_ver,
+                                                      workspace=wk.workspace, status=wk.status))
+        wk.draft_cache.kv_len = wk.len_draft[s0, 0]
+        nat_b2b = graph_call_us(lambda: w.draft_attn_full(wk.p, wk.q_draft[s0][0], wk.draft_cache, out=wk.o_draft,
+                                                          lse=wk.l_draft, workspace=wk.workspace,
+                                                          status=wk.status))
+        b2b = {"verify_us": ver_b2b, "verify_gbs": ver_bytes / (ver_b2b * 1e-6) / 1e9,
+               "draft_native_us": nat_b2b, "draft_native_gbs": nat_bytes / (nat_b2b * 1e-6) / 1e9}
+
     # the windowed draft at 32K, 128K and 1M tokens of context (one sequence,
     # the ring in the state it has at that length): its time must not grow
     # with the context
@@ -1099,6 +1118,7 @@ def main():
             "draft_native_us": k_nat["draft"],
             "draft_windowed_us": k_win["draft"],
             "draft_windowed_paged_us": win_paged_us,
+            "back_to_back": b2b,
             "draft_windowed_us_by_context": flat,
             "draft_windowed_spread_by_context": ((max(flat.values()) - min(flat.values())) / statistics.median(
                 flat.values())) if flat else None,
