@@ -240,6 +240,25 @@ wmtp_status wmtp_verify_attn(const wmtp_params* params, int32_t batch, int32_t n
                              size_t* workspace_bytes, int32_t* status_word, void* stream);
 
 /*
+ * wmtp_verify_attn_append -- wmtp_paged_write of the num_q new tokens at
+ * positions kv_len[b]-num_q .. kv_len[b]-1, then wmtp_verify_attn, in one
+ * call.  Source: howtospark case study, Method (a verify layer appends its
+ * gamma+1 tokens and attends over them); the fusion is this library's.
+ * On the tcgen05 verify path (head_dim 256, 2 <= num_q, 9..128 rows per KV
+ * head) the verify kernel writes each new row itself, with plain stores
+ * ordered before the bulk copy that loads its tile, so no separate write is
+ * launched; other shapes launch the paged write in front of the verify.
+ *   k_new, v_new: [batch][num_q][Hkv][D] bf16, 16-byte aligned, not NULL
+ *   when workspace is given.  Pages and lengths are checked as in
+ *   wmtp_paged_write (a new row on a page outside the pool is not written and
+ *   sets WMTP_DEV_PAGE_OOB).  Everything else as wmtp_verify_attn.
+ */
+wmtp_status wmtp_verify_attn_append(const wmtp_params* params, int32_t batch, int32_t num_q, const void* q,
+                                    const void* k_new, const void* v_new, const wmtp_paged_kv* kv, void* out,
+                                    int32_t out_fp32, float* lse_out, void* workspace, size_t* workspace_bytes,
+                                    int32_t* status_word, void* stream);
+
+/*
  * wmtp_verify_attn_slice -- verify attention over one slice of each
  * sequence's context (context parallelism).
  * Not on the pages as such: the pages verify on one GPU.  A sequence whose

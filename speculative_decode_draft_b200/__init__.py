@@ -23,6 +23,7 @@ from .api import (  # noqa: F401
     selftest_wait,
     splitkv_combine,
     verify_attn,
+    verify_attn_append,
     workspace_bytes,
 )
 

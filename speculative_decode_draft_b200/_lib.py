@@ -37,6 +37,7 @@ EXPORTS = (
     "wmtp_ring_append",
     "wmtp_ring_reset",
     "wmtp_verify_attn",
+    "wmtp_verify_attn_append",
     "wmtp_verify_attn_slice",
     "wmtp_splitkv_combine",
     "wmtp_paged_write",
@@ -141,6 +142,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.wmtp_verify_attn.restype = c_int32
     lib.wmtp_verify_attn.argtypes = [PP, c_int32, c_int32, c_void_p, PK, c_void_p, c_int32, c_void_p,
                                      c_void_p, sz, i32p, c_void_p]
+    lib.wmtp_verify_attn_append.restype = c_int32
+    lib.wmtp_verify_attn_append.argtypes = [PP, c_int32, c_int32, c_void_p, c_void_p, c_void_p, PK, c_void_p,
+                                            c_int32, c_void_p, c_void_p, sz, i32p, c_void_p]
     lib.wmtp_verify_attn_slice.restype = c_int32
     lib.wmtp_verify_attn_slice.argtypes = [PP, c_int32, c_int32, c_void_p, PK, c_void_p, c_void_p, c_int32,
                                            c_void_p, c_void_p, sz, i32p, c_void_p]

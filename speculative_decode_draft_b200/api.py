@@ -228,6 +228,29 @@ def verify_attn(p: L.Params, q: torch.Tensor, cache: PagedCache, *, out_fp32: bo
                           workspace, status)
 
 
+def verify_attn_append(p: L.Params, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                       cache: PagedCache, *, out_fp32: bool = True, out=None, lse=None, workspace=None,
+                       status=None, stream=None):
+    """``paged_write`` of ``k_new/v_new [B, num_q, Hkv, D]`` at the last num_q
+    positions of each sequence (``cache.kv_len`` includes them), then
+    ``verify_attn``, in one call (``wmtp_verify_attn_append``)."""
+    _need(q, BF16, "q")
+    _need(k_new, BF16, "k_new", q.device)
+    _need(v_new, BF16, "v_new", q.device)
+    B, Qn, Hq, D = q.shape
+    if tuple(k_new.shape[:2]) != (B, Qn) or k_new.shape != v_new.shape:
+        raise ValueError(f"k_new/v_new must be [B, num_q, Hkv, D] = [{B}, {Qn}, ...], got {tuple(k_new.shape)}")
+    desc = cache.desc()
+    st = _stream(stream)
+
+    def call(fn, o, l, ws, _unused, size, stat):
+        live = ws is not None
+        return fn(byref(p), B, Qn, q.data_ptr() if live else None, k_new.data_ptr() if live else None,
+                  v_new.data_ptr() if live else None, byref(desc), o, int(out_fp32), l, ws, size, stat, st)
+    return _run_attention("wmtp_verify_attn_append", call, (B, Qn, Hq, D), q.device, out_fp32, out, lse,
+                          workspace, status)
+
+
 def draft_attn_windowed(p: L.Params, q: torch.Tensor, ring: Ring, *, out_fp32: bool = True, out=None,
                         lse=None, workspace=None, status=None, stream=None):
     """Windowed-MTP draft attention over the rings: q ``[B, Hq, D]`` bf16."""

@@ -99,6 +99,13 @@ struct DecodeArgs {
   int nsplit;
   float scale_log2;  // sm_scale * log2(e)
   int32_t* status;
+  // tcgen05 verify only, or NULL: the num_q new tokens' K/V ([B][num_q][Hkv][D]
+  // bf16), written into the pools (k_pool_w, v_pool_w: [num_pages][Hkv][P][D])
+  // at positions kv_len - num_q .. kv_len - 1 before their tiles are loaded
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pool_w;
+  __nv_bfloat16* v_pool_w;
 };
 
 __device__ __forceinline__ void set_status(int32_t* status, int bits) {

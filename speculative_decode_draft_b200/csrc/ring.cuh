@@ -183,11 +183,14 @@ __global__ void ring_reset_kernel(RingArgs r) {
 }
 
 // Write n_new tokens per sequence into a paged cache: grid (n_new, batch).
+// `len_end`: NULL, or [batch] lengths whose last n_new positions are written
+// (pos0 then unused): the append in front of a verify whose new tokens end
+// the sequence.
 __global__ void paged_write_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool, int num_pages,
                                    const int32_t* __restrict__ page_table, int max_pages, int P,
                                    int Hkv, int D, const int32_t* __restrict__ pos0, int n_new,
                                    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
-                                   int32_t* status) {
+                                   int32_t* status, const int32_t* __restrict__ len_end) {
   const int j = blockIdx.x;
   const int b = blockIdx.y;
   // launched as a programmatic dependent: wait (unconditionally, before any
@@ -195,7 +198,7 @@ __global__ void paged_write_kernel(uint4* __restrict__ k_pool, uint4* __restrict
   // attention kernel behind it get scheduled
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int p = pos0[b] + j;
+  const int p = (len_end != nullptr ? len_end[b] - n_new : pos0[b]) + j;
   if (p < 0 || p >= max_pages * P) {
     if (threadIdx.x == 0) set_status(status, kDevLenOob);
     return;

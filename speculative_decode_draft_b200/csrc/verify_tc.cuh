@@ -304,6 +304,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::tma_load_3d(dst + c * Plan::kChunkBytes + j * box_rows * 128, tmap, fb, c * 64, ys[j], zs[j], pol);
     }
   };
+  // The fused append: the new rows (positions n_tok - num_q .. n_tok - 1)
+  // that fall in this CTA's tiles go into the pools before any of its tiles
+  // is loaded -- K by warp 0, V by warp 3, all lanes, every load of a lane
+  // before its stores.  Each lane orders its stores before the async proxy,
+  // then the warp converges before lane 0 issues a bulk copy.  Only the CTA
+  // that loads a tile reads its new rows.  A row on a page outside the pool
+  // is skipped (the tile's loads raise WMTP_DEV_PAGE_OOB).
+  if (a.k_new != nullptr && (warp == 0 || warp == kVWarp) && my_tiles > 0) {
+    const int new_lo = n_tok - a.num_q;
+    const int lo = max(new_lo, t_begin * kTileTokens), hi = min(n_tok, t_end * kTileTokens);
+    if (lo < hi) {
+      constexpr int kUnits = D / 8;  // 16-byte units of a row
+      const uint4* src = reinterpret_cast<const uint4*>(is_k ? a.k_new : a.v_new);
+      uint4* pool = reinterpret_cast<uint4*>(is_k ? a.k_pool_w : a.v_pool_w);
+      const int n_units = (hi - lo) * kUnits;
+      // four units a lane per round: every load of the round before its stores
+      for (int u0 = 0; u0 < n_units; u0 += 4 * 32) {
+        uint4 val[4];
+        size_t dst[4];
+        bool ok[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int u = u0 + i * 32 + lane;
+          ok[i] = u < n_units;
+          if (!ok[i]) continue;
+          const int pos = lo + u / kUnits, c = u % kUnits;
+          const int pg = a.page_table[static_cast<size_t>(b) * a.max_pages + pos / a.page_size];
+          ok[i] = pg >= 0 && pg < a.num_pages;
+          dst[i] = ((static_cast<size_t>(pg) * a.Hkv + kvh) * a.page_size + pos % a.page_size) * kUnits + c;
+          val[i] = src[((static_cast<size_t>(b) * a.num_q + (pos - new_lo)) * a.Hkv + kvh) * kUnits + c];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (ok[i]) pool[dst[i]] = val[i];
+      }
+      ptx::fence_proxy_async_global();
+    }
+    __syncwarp();
+  }
   // tile 0 of each ring goes out before the block-wide barrier (the
   // producers initialised their own barriers), and the page-table lines of
   // the next tiles head for L2

@@ -340,20 +340,35 @@ wmtp_status run_attention(const wmtp_params* p, int B, int num_q, const void* q,
   a.scale_log2 = scale_log2(p);
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_lse);
-  if (tc)
-    s = launch_verify_tc(*tk, *tv, a, B, st);
-  else
+  if (tc) {
+    s = launch_verify_tc(*tk, *tv, a, B, st);  // writes a.k_new / a.v_new itself
+  } else {
+    if (a.k_new != nullptr) {
+      // the mma.sync verify's shapes: the append as its own launch in front
+      s = launch_plain(true, paged_write_kernel, dim3(num_q, B), dim3(128), st, reinterpret_cast<uint4*>(a.k_pool_w),
+                       reinterpret_cast<uint4*>(a.v_pool_w), a.num_pages, a.page_table, a.max_pages, a.page_size,
+                       a.Hkv, D, static_cast<const int32_t*>(nullptr), num_q,
+                       reinterpret_cast<const uint4*>(a.k_new), reinterpret_cast<const uint4*>(a.v_new), a.status,
+                       a.kv_len);
+      if (s != WMTP_OK) return s;
+      a.k_new = a.v_new = nullptr;
+    }
     s = launch_decode<RING>(D, NT, *tk, *tv, a, B, st);
+  }
   if (s != WMTP_OK) return s;
   return launch_combine(static_cast<int>(rows_total), D, pl.nsplit, a.part_o, a.part_lse, out, out_fp32,
                         lse_out, st, true);
 }
 
 // `window`: attend only the sink + window positions of the pages (num_q 1).
+// `k_new`, `v_new` (verify only): the num_q new tokens' K/V, written at the
+// sequence's last num_q positions before they are read -- inside the tcgen05
+// verify kernel, else by a paged write launched in front of it.
 wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, const void* q,
                             const wmtp_paged_kv* kv, void* out, int32_t out_fp32, float* lse_out,
                             void* workspace, size_t* workspace_bytes, int32_t* status_word, void* stream,
-                            bool window = false, const int32_t* q_pos0 = nullptr) {
+                            bool window = false, const int32_t* q_pos0 = nullptr, const void* k_new = nullptr,
+                            const void* v_new = nullptr) {
   wmtp_status s = check_params(p, num_q);
   if (s != WMTP_OK) return s;
   if (window && (num_q != 1 || p->sinks < 0 || p->window < 1)) return WMTP_ERR_INVALID_ARG;
@@ -400,6 +415,13 @@ wmtp_status paged_attention(const wmtp_params* p, int32_t batch, int32_t num_q, 
   a.q_pos0 = q_pos0;
   a.sinks = p->sinks;
   a.window = p->window;
+  if (k_new != nullptr && workspace != nullptr) {
+    if (!aligned(k_new, 16) || !aligned(v_new, 16)) return WMTP_ERR_INVALID_ARG;
+    a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    a.k_pool_w = static_cast<__nv_bfloat16*>(kv->k_pool);
+    a.v_pool_w = static_cast<__nv_bfloat16*>(kv->v_pool);
+  }
   return run_attention<false>(p, batch, num_q, q, &tk, &tv, a, max_tiles, out, out_fp32, lse_out, workspace,
                               workspace_bytes, static_cast<cudaStream_t>(stream), ready);
 }
@@ -494,6 +516,15 @@ wmtp_status wmtp_verify_attn(const wmtp_params* params, int32_t batch, int32_t n
                          status_word, stream);
 }
 
+wmtp_status wmtp_verify_attn_append(const wmtp_params* params, int32_t batch, int32_t num_q, const void* q,
+                                    const void* k_new, const void* v_new, const wmtp_paged_kv* kv, void* out,
+                                    int32_t out_fp32, float* lse_out, void* workspace, size_t* workspace_bytes,
+                                    int32_t* status_word, void* stream) {
+  if (workspace != nullptr && batch > 0 && (k_new == nullptr || v_new == nullptr)) return WMTP_ERR_INVALID_ARG;
+  return paged_attention(params, batch, num_q, q, kv, out, out_fp32, lse_out, workspace, workspace_bytes,
+                         status_word, stream, false, nullptr, k_new, v_new);
+}
+
 wmtp_status wmtp_draft_attn_windowed(const wmtp_params* params, const void* q, const wmtp_ring* ring,
                                      void* out, int32_t out_fp32, float* lse_out, void* workspace,
                                      size_t* workspace_bytes, int32_t* status_word, void* stream) {
@@ -584,7 +615,7 @@ wmtp_status wmtp_paged_write(const wmtp_params* params, int32_t batch, const wmt
                       static_cast<uint4*>(kv->k_pool), static_cast<uint4*>(kv->v_pool), kv->num_pages,
                       kv->page_table, kv->max_pages, params->page_size, params->num_heads_kv, params->head_dim,
                       pos0, n_new, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-                      status_word);
+                      status_word, static_cast<const int32_t*>(nullptr));
 }
 
 }  // extern "C"
