@@ -167,3 +167,20 @@ def test_selftest_wait_rejects_misaligned_pointers(lib):
     assert lib.wmtp_selftest_wait(0, None, 4, None) == L.WMTP_ERR_INVALID_ARG
     assert lib.wmtp_selftest_wait(0, 2, None, None) == L.WMTP_ERR_INVALID_ARG
     assert L.WAIT_LIMIT_CYCLES == 4_000_000_000
+
+
+def test_verify_append_rejects_missing_new_tokens(lib):
+    # checked before anything is launched, so this runs without a GPU
+    desc = L.PagedKVDesc(None, None, 8, None, 8, None)
+    ws = ctypes.create_string_buffer(512)
+    have = c_size_t(256)
+    base = ctypes.addressof(ws) // 256 * 256 + 256
+    for k_new, v_new in ((None, base), (base, None), (None, None)):
+        assert lib.wmtp_verify_attn_append(byref(_p()), 1, 4, None, k_new, v_new, byref(desc), None, 1, None,
+                                           base, byref(have), None, None) == L.WMTP_ERR_INVALID_ARG
+    # the size query needs no new tokens, and rejects what wmtp_verify_attn rejects
+    size = c_size_t(0)
+    assert lib.wmtp_verify_attn_append(byref(_p()), 1, 17, None, None, None, byref(desc), None, 1, None, None,
+                                       byref(size), None, None) == L.WMTP_ERR_UNSUPPORTED  # 136 rows
+    assert lib.wmtp_verify_attn_append(byref(_p()), 0, 4, None, None, None, byref(desc), None, 1, None, None,
+                                       byref(size), None, None) == 0  # empty batch
