@@ -349,9 +349,15 @@ class Workload:
 
     # -- kernel launches of one step (for gpu_launches)
     def launches_per_step(self, arm: str) -> int:
-        if arm == "windowed":
-            return self.gamma * (1 + 2) + self.L * (1 + 2) + 1
-        return self.gamma * (1 + 2) + self.L * (1 + 2)
+        """Library kernels one decode step launches: per draft an append (ring
+        or paged write), the attention and its combine; per verify layer the
+        verify (which writes its new tokens itself on the tcgen05 path, else
+        after a paged write) and its combine; the windowed arm's final ring
+        append (accept / rollback)."""
+        rows = (self.gamma + 1) * self.Hq // self.Hkv
+        tc = self.D == 256 and self.gamma + 1 >= 2 and 9 <= rows <= 128
+        n = self.gamma * 3 + self.L * (2 if tc else 3)
+        return n + 1 if arm == "windowed" else n
 
     # -- one decode step; `ev` collects (kind, start_event, end_event)
     # names of the per-step input tensors (first dimension: the step)
@@ -1139,7 +1145,7 @@ def main():
                                "call (verify_tc_kernel + its split-KV combine)",
                      "algorithmic_bytes": ver_bytes, "peak_source": peak_src},
         "e2e": e2e,
-        "gpu_launches": wk.launches_per_step("windowed") * args.steps,
+        "gpu_launches": (wk.launches_per_step("windowed") + wk.launches_per_step("native")) * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu,
     }

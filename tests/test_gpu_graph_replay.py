@@ -4,7 +4,8 @@ same step launched eagerly.
 The bench times steps as graph replays, and the attention kernels are
 launched as programmatic dependents of the previous stream work; this checks
 that the captured dependencies (ring append -> windowed draft, paged write ->
-verify, attention -> combine) order the work exactly as stream order does.
+verify, attention -> combine, and the verify that writes its own new tokens)
+order the work exactly as stream order does.
 """
 
 import pytest
@@ -36,7 +37,8 @@ def test_graph_replay_matches_eager_step():
     i32 = dict(dtype=torch.int32, device=DEV)
     draft = synth.paged_kv(21, 1, Hkv, D, P, [n0], cap, True, True, device=DEV)
     ver = synth.paged_kv(22, 1, Hkv, D, P, [n0], cap, True, True, device=DEV)
-    dcache, vcache = cache_of(draft), cache_of(ver)
+    ver2 = synth.paged_kv(27, 1, Hkv, D, P, [n0], cap, True, True, device=DEV)
+    dcache, vcache, vcache2 = cache_of(draft), cache_of(ver), cache_of(ver2)
     ring = w.Ring.allocate(p, 1, DEV)
     k, v = synth.dense_from_paged(draft, 0, n0)
     w.ring_append(p, ring, k[None].contiguous(), v[None].contiguous(), torch.tensor([n0], **i32))
@@ -58,6 +60,7 @@ def test_graph_replay_matches_eager_step():
     l_n = torch.empty_like(l_w)
     o_v = torch.empty(1, gamma + 1, Hq, D, dtype=torch.float32, device=DEV)
     l_v = torch.empty(1, gamma + 1, Hq, dtype=torch.float32, device=DEV)
+    o_v2, l_v2 = torch.empty_like(o_v), torch.empty_like(l_v)
     ws = torch.empty(max(w.workspace_bytes("full", p, 1, max_pages=draft.max_pages),
                          w.workspace_bytes("verify", p, 1, num_q=gamma + 1, max_pages=ver.max_pages),
                          w.workspace_bytes("windowed", p, 1)), dtype=torch.uint8, device=DEV)
@@ -73,17 +76,21 @@ def test_graph_replay_matches_eager_step():
         w.paged_write(p, vcache, pos_v, kv_, vv_, status=status)
         vcache.kv_len = len_v
         w.verify_attn(p, qv, vcache, out=o_v, lse=l_v, workspace=ws, status=status)
+        # a second layer with the append fused into the verify call (rewriting
+        # the same rows on replay leaves the pool unchanged)
+        vcache2.kv_len = len_v
+        w.verify_attn_append(p, qv, kv_, vv_, vcache2, out=o_v2, lse=l_v2, workspace=ws, status=status)
         w.ring_append(p, ring, kd[:, :1], vd[:, :1], none, truncate_to=trunc, status=status)
 
     snap = [t.clone() for t in (ring.k, ring.v, ring.tags, ring.len, ring.committed)]
     step()
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    eager = [t.clone() for t in (o_w, l_w, o_n, l_n, o_v, l_v, ring.k, ring.v, ring.tags, ring.len,
+    eager = [t.clone() for t in (o_w, l_w, o_n, l_n, o_v, l_v, o_v2, l_v2, ring.k, ring.v, ring.tags, ring.len,
                                  ring.committed)]
     for dst, src in zip((ring.k, ring.v, ring.tags, ring.len, ring.committed), snap):
         dst.copy_(src)
-    for t in (o_w, l_w, o_n, l_n, o_v, l_v):
+    for t in (o_w, l_w, o_n, l_n, o_v, l_v, o_v2, l_v2):
         t.zero_()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
@@ -92,8 +99,9 @@ def test_graph_replay_matches_eager_step():
     g.replay()
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    replay = (o_w, l_w, o_n, l_n, o_v, l_v, ring.k, ring.v, ring.tags, ring.len, ring.committed)
+    replay = (o_w, l_w, o_n, l_n, o_v, l_v, o_v2, l_v2, ring.k, ring.v, ring.tags, ring.len, ring.committed)
     for name, a, b in zip(("windowed out", "windowed lse", "native out", "native lse", "verify out",
-                           "verify lse", "ring k", "ring v", "ring tags", "ring len", "ring committed"),
+                           "verify lse", "fused verify out", "fused verify lse", "ring k", "ring v", "ring tags",
+                           "ring len", "ring committed"),
                           eager, replay):
         assert torch.equal(a, b), f"graph replay differs from eager launches: {name}"
