@@ -600,11 +600,12 @@ def cores_used():
 # roofline.traffic is null.
 VERIFY_TRAFFIC = {
     "sources": ("speculative_decode_draft_b200/csrc/verify_tc.cuh", "speculative_decode_draft_b200/csrc/ptx.cuh"),
-    "sha256": "bb3fb9a0c48599da0a267e0d604f2cf4f100b245e4ba90162f207ba335c5dd02",
-    "captured_on": "128k: verify_tc_kernel<3, 3, 64> with the fused append, 148 CTAs x 384 threads",
+    "sha256": "0aa88727134350119405ddb7b47311b7bcd6131ac7c235e4beeac024cf25ef9f",
+    "captured_on": "128k: verify_tc_kernel<3, 3, 64> with the fused append and P_lo in the spare lanes, "
+                   "148 CTAs x 384 threads",
     "tokens": 131076,
-    "read_bytes": 268722176,
-    "write_bytes": 3541760,
+    "read_bytes": 268724224,
+    "write_bytes": 5498112,
 }
 
 

@@ -265,6 +265,16 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t* v) 
       : "memory");
 }
 
+// One 16x128b.x4 store (16 columns, 8 registers: v[2r] to lane t/4 and
+// v[2r + 1] to lane t/4 + 8, column 4r + t%4) and its wait.
+__device__ __forceinline__ void tmem_st_16x128b_x4(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+
 // Two 16x128b.x4 stores (16 columns, 8 registers each: the first four
 // repetitions of the x8 layout) and one wait for both.
 __device__ __forceinline__ void tmem_st_16x128b_x4_pair(uint32_t taddr0, const uint32_t* v, uint32_t taddr1,

@@ -16,8 +16,11 @@
 //   M = 64:  columns 0..191 S / P x 3, columns 256..511 O
 //   M = 128: columns 0..127 Q (bf16 pairs), 128..255 S / P x 2, 256..511 O
 // An S buffer holds a tile's fp32 scores; after the softmax its columns 0..31
-// hold P_hi and 32..63 P_lo as bf16 pairs (P = hi + lo).  O is the fp32
-// output accumulator, 256 head dims.  QK(k) may overwrite buffer k % NB only
+// hold P_hi and 32..63 P_lo as bf16 pairs (P = hi + lo).  A block of up to
+// 32 rows uses only half of the M = 64 lanes, so there P_lo goes to the
+// row's spare lane (M row + 8) in columns 0..31 and one MMA per 16 tokens
+// takes both; O's spare-lane rows then hold the P_lo products, added to
+// their row at the end.  O is the fp32 output accumulator, 256 head dims.  QK(k) may overwrite buffer k % NB only
 // once PV(k - NB) has read it, so with three buffers the QK of a tile no
 // longer waits for the PV of the tile just before the previous one.
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
@@ -254,6 +257,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int t_begin = min(split * tps, ntiles);
   const int t_end = min(t_begin + tps, ntiles);
   const int my_tiles = t_end - t_begin;
+  // Blocks of up to 32 rows fill only the sub-row j = 0 lanes of an M = 64
+  // MMA (rows 16 (r % 4) + r / 4 < 8 of each quadrant's sixteen).  P_lo of a
+  // row then sits in the row's spare lane (+8), so P_hi and P_lo go through
+  // one MMA per 16 tokens, and O's spare-lane rows hold the P_lo products,
+  // which the epilogue adds to their row.
+  const bool stacked = QS && a.rows <= 32;
 
   // ---- producers: warp 0 loads K tiles, warp 3 V tiles (lane 0 each), each
   // into its own ring.  Tile k of a ring goes to stage k % depth.
@@ -421,7 +430,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // O += P(k) V(k) for every tile, issued by its own lane: a single lane
   // issues a small tcgen05.mma only every ~66 cycles, so the QK and PV
   // streams run from two lanes and overlap in the tensor pipe.  Per 16
-  // tokens two MMAs: P_hi V and P_lo V.  The first MMA of a run starts a
+  // tokens two MMAs, P_hi V and P_lo V, or one for a stacked block (P_hi and
+  // P_lo in the same columns, different lanes).  The first MMA of a run starts a
   // fresh accumulation (the softmax threads have folded the previous run).
   if (warp == kPvWarp) {
     if (lane == 0 && my_tiles > 0) {
@@ -441,7 +451,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // 16 tokens = 8 columns of bf16 pairs; V rows 16 kk .. 16 kk + 15
           const uint64_t bd = vd + (static_cast<uint32_t>(kk * 2048) >> 4);
           tc::mma_ts(tmem_base + kColO, p_tmem + 8 * kk, bd, kIdescPV, kk > 0 ? 1u : fresh);
-          tc::mma_ts(tmem_base + kColO, p_tmem + 32 + 8 * kk, bd, kIdescPV, 1u);
+          if (!stacked) tc::mma_ts(tmem_base + kColO, p_tmem + 32 + 8 * kk, bd, kIdescPV, 1u);
         }
         tc::commit(bar_v_empty + 8 * (k % VS));
         tc::commit(bar_pv_done + 8 * (k % NB));
@@ -657,8 +667,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               for (int r = 0; r < 8; ++r) {
                 float2* g = reinterpret_cast<float2*>(d + 8 * r);
                 const float2 old = have_g[h][j] ? *g : make_float2(0.f, 0.f);
-                *g = make_float2(old.x * gs[j] + __uint_as_float(o[4 * r + 2 * j]),
-                                 old.y * gs[j] + __uint_as_float(o[4 * r + 2 * j + 1]));
+                float o0 = __uint_as_float(o[4 * r + 2 * j]), o1 = __uint_as_float(o[4 * r + 2 * j + 1]);
+                if (stacked) {  // j = 0: add the spare lane's P_lo products
+                  o0 += __uint_as_float(o[4 * r + 2]);
+                  o1 += __uint_as_float(o[4 * r + 3]);
+                }
+                *g = make_float2(old.x * gs[j] + o0, old.y * gs[j] + o1);
               }
             }
           }
@@ -804,13 +818,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                   for (int e = 0; e < 2; ++e)
-                    o[4 * r + 2 * j + e] = __float_as_uint(__uint_as_float(o[4 * r + 2 * j + e]) * alpha[j]);
+                    o[4 * r + 2 * j + e] =
+                        __float_as_uint(__uint_as_float(o[4 * r + 2 * j + e]) * (stacked ? alpha[0] : alpha[j]));
               tc::tmem_st_16x256b_x8(o_addr(h, cb), o);
             }
           }
           // P = 2^(x - m_ref) as bf16 hi + lo pairs: token pair
           // 16 half + 4 r + lane % 4 of the tile, back into the S columns
-          // (P_hi in columns 0..31, P_lo in 32..63)
+          // (P_hi in columns 0..31, P_lo in 32..63; in a stacked block P_lo
+          // in the row's spare lane, columns 0..31)
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             if (!any_r[h][j]) continue;
@@ -827,7 +843,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         const uint32_t s_addr = s_addr_of(h, sb);
-        tc::tmem_st_16x128b_x4_pair(s_addr + 16 * half, ph, s_addr + 32 + 16 * half, pl);
+        if (stacked) {
+          // P_hi in the row's lane, P_lo in its spare lane, same columns
+          uint32_t pk[8];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            pk[2 * r] = ph[2 * r];
+            pk[2 * r + 1] = pl[2 * r];
+          }
+          tc::tmem_st_16x128b_x4(s_addr + 16 * half, pk);
+        } else {
+          tc::tmem_st_16x128b_x4_pair(s_addr + 16 * half, ph, s_addr + 32 + 16 * half, pl);
+        }
       }
       if (failed) break;
 
@@ -902,8 +929,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int r = 0; r < 8; ++r) {
             float2* g = reinterpret_cast<float2*>(d + 8 * r);
             const float2 old = (have_g[h][j] && !failed) ? *g : make_float2(0.f, 0.f);
-            *g = make_float2((old.x * gs[j] + __uint_as_float(o[4 * r + 2 * j])) * inv[j],
-                             (old.y * gs[j] + __uint_as_float(o[4 * r + 2 * j + 1])) * inv[j]);
+            float o0 = __uint_as_float(o[4 * r + 2 * j]), o1 = __uint_as_float(o[4 * r + 2 * j + 1]);
+            if (stacked) {  // j = 0: add the spare lane's P_lo products
+              o0 += __uint_as_float(o[4 * r + 2]);
+              o1 += __uint_as_float(o[4 * r + 3]);
+            }
+            *g = make_float2((old.x * gs[j] + o0) * inv[j], (old.y * gs[j] + o1) * inv[j]);
           }
         }
       }
