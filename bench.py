@@ -372,8 +372,9 @@ class Workload:
     def step(self, s: int, arm: str, ev=None, inputs=None, external_events: bool = False, outputs=None):
         """One decode step.  ``inputs`` (a dict like ``step_inputs``) replaces
         the resident inputs of step ``s``; ``outputs`` (``{"draft": [gamma,
-        ...], "verify": [L, ...]}``, e.g. pinned host buffers) receives every
-        attention output of the step.  With ``ev`` one draft call and one
+        ...], "verify": [L, ...]}`` device tensors) are written by the
+        attention calls themselves in place of the resident output buffers.
+        With ``ev`` one draft call and one
         verify call of the step (draft s mod gamma, layer s mod L) are
         bracketed by an event pair: an event node between two kernels ends the
         second one's programmatic overlap with the first, so the other calls
@@ -384,6 +385,8 @@ class Workload:
             return torch.cuda.Event(external=external_events, **kw)
         x = inputs if inputs is not None else self.step_inputs(s)
         ev_all = ev
+        o_draft = (lambda j: outputs["draft"][j]) if outputs is not None else (lambda j: self.o_draft)
+        o_ver = (lambda l: outputs["verify"][l]) if outputs is not None else (lambda l: self.o_ver)
         for j in range(self.gamma):
             ev = ev_all if j == s % self.gamma else None
             if arm == "windowed":
@@ -392,7 +395,7 @@ class Workload:
                 a = E(enable_timing=True) if ev is not None else None
                 if a is not None:
                     a.record()
-                w.draft_attn_windowed(self.p, x["q_draft"][j], self.ring, out=self.o_draft, lse=self.l_draft,
+                w.draft_attn_windowed(self.p, x["q_draft"][j], self.ring, out=o_draft(j), lse=self.l_draft,
                                       workspace=self.workspace, status=self.status)
             else:
                 self.draft_cache.kv_len = x["len_draft"][j]
@@ -401,14 +404,12 @@ class Workload:
                 a = E(enable_timing=True) if ev is not None else None
                 if a is not None:
                     a.record()
-                w.draft_attn_full(self.p, x["q_draft"][j], self.draft_cache, out=self.o_draft, lse=self.l_draft,
+                w.draft_attn_full(self.p, x["q_draft"][j], self.draft_cache, out=o_draft(j), lse=self.l_draft,
                                   workspace=self.workspace, status=self.status)
             if ev is not None:
                 bnd = E(enable_timing=True)
                 bnd.record()
                 ev.append(("draft", a, bnd))
-            if outputs is not None:
-                outputs["draft"][j].copy_(self.o_draft, non_blocking=True)
         for l in range(self.L):
             ev = ev_all if l == s % self.L else None
             c = self.caches[l]
@@ -418,14 +419,12 @@ class Workload:
                 a.record()
             # the layer's gamma+1 new tokens are written by the verify call
             # itself (positions len_ver - gamma - 1 = pos_ver ..)
-            w.verify_attn_append(self.p, x["q_ver"][l], x["k_ver"][l], x["v_ver"][l], c, out=self.o_ver,
+            w.verify_attn_append(self.p, x["q_ver"][l], x["k_ver"][l], x["v_ver"][l], c, out=o_ver(l),
                                  lse=self.l_ver, workspace=self.workspace, status=self.status)
             if ev is not None:
                 bnd = E(enable_timing=True)
                 bnd.record()
                 ev.append(("verify", a, bnd))
-            if outputs is not None:
-                outputs["verify"][l].copy_(self.o_ver, non_blocking=True)
         if arm == "windowed":
             w.ring_append(self.p, self.ring, x["k_bonus"], x["v_bonus"], x["n_bonus"],
                           truncate_to=x["trunc_to"], status=self.status)
@@ -963,19 +962,37 @@ def main():
 
     # ---------------- end to end: host buffers, copies inside the timed region
     # Every step's inputs (queries, new K/V, lengths, positions, rollback
-    # targets, bonus counts) start in pinned host memory and are copied in;
-    # every attention output of the step is copied back out.
+    # targets, bonus counts) start in pinned host memory and go to the device
+    # in one copy; the attention calls write every output of the step into a
+    # device staging buffer, which goes back to pinned host memory in one copy.
     e2e = None
     if not args.no_e2e:
-        pin = dict(pin_memory=True)
         steps = range(args.warmup, args.warmup + args.steps)
-        host_in = {s: {k: torch.empty(v.shape, dtype=v.dtype, **pin).copy_(v) for k, v in wk.step_inputs(s).items()}
-                   for s in steps}
-        dev_in = {k: torch.empty_like(v) for k, v in wk.step_inputs(args.warmup).items()}
-        outs = {"draft": torch.empty((wk.gamma,) + tuple(wk.o_draft.shape), dtype=torch.float32, **pin),
-                "verify": torch.empty((wk.L,) + tuple(wk.o_ver.shape), dtype=torch.float32, **pin)}
-        h2d = sum(v.numel() * v.element_size() for v in dev_in.values())
-        d2h = sum(v.numel() * v.element_size() for v in outs.values())
+        proto = wk.step_inputs(args.warmup)
+        offs, off = {}, 0
+        for k, v in proto.items():  # 256-byte aligned slots of one flat buffer
+            offs[k] = off
+            off += -(-v.numel() * v.element_size() // 256) * 256
+        dev_flat = torch.empty(off, dtype=torch.uint8, device=dev)
+
+        def views(flat):
+            return {k: flat[offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+                    for k, v in proto.items()}
+        host_in = {}
+        for st_ in steps:
+            flat = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+            for k, v in views(flat).items():
+                v.copy_(wk.step_inputs(st_)[k])
+            host_in[st_] = flat
+        dev_in = views(dev_flat)
+        n_d = wk.o_draft.numel()
+        n_v = wk.o_ver.numel()
+        out_flat = torch.empty(wk.gamma * n_d + wk.L * n_v, dtype=torch.float32, device=dev)
+        outs = {"draft": out_flat[:wk.gamma * n_d].view((wk.gamma,) + tuple(wk.o_draft.shape)),
+                "verify": out_flat[wk.gamma * n_d:].view((wk.L,) + tuple(wk.o_ver.shape))}
+        host_out = {st_: torch.empty_like(out_flat, device="cpu", pin_memory=True) for st_ in steps}
+        h2d = off
+        d2h = out_flat.numel() * out_flat.element_size()
         wk.restore_ring(ring_after_warmup)
         barrier(world)
         torch.cuda.synchronize()
@@ -983,17 +1000,17 @@ def main():
         en = torch.cuda.Event(enable_timing=True)
         st.record()
         for s in steps:
-            for k, v in dev_in.items():
-                v.copy_(host_in[s][k], non_blocking=True)
+            dev_flat.copy_(host_in[s], non_blocking=True)
             wk.step(s, "windowed", inputs=dev_in, outputs=outs)
+            host_out[s].copy_(out_flat, non_blocking=True)
         en.record()
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(st.elapsed_time(en), world)
         e2e = {"value": whole_job_us_per_step(ms_e2e, args.steps, world), "unit": "us/step",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "arm": "windowed",
-               "path": "public Python API (eager launches), inputs copied from pinned host memory and outputs "
-                       "copied back each step"}
-        del host_in, dev_in, outs
+               "path": "public Python API (eager launches); each step's inputs copied in from pinned host memory "
+                       "in one transfer and its attention outputs copied back to pinned host memory in one"}
+        del host_in, dev_in, outs, host_out, dev_flat, out_flat
 
     torch.cuda.synchronize()
     status = int(wk.status.item())
