@@ -20,9 +20,10 @@
 // 32 rows uses only half of the M = 64 lanes, so there P_lo goes to the
 // row's spare lane (M row + 8) in columns 0..31 and one MMA per 16 tokens
 // takes both; O's spare-lane rows then hold the P_lo products, added to
-// their row at the end.  O is the fp32 output accumulator, 256 head dims.  QK(k) may overwrite buffer k % NB only
-// once PV(k - NB) has read it, so with three buffers the QK of a tile no
-// longer waits for the PV of the tile just before the previous one.
+// their row at the end.  O is the fp32 output accumulator, 256 head dims.
+// QK(k) may overwrite buffer k % NB only once PV(k - NB) has read it, so
+// with three buffers the QK of a tile no longer waits for the PV of the
+// tile just before the previous one.
 // Row r of the block sits in TMEM lane 32 (r % 4) + r / 4 (M row
 // 16 (r % 4) + r / 4 for M=64, 32 (r % 4) + r / 4 for M=128), so the rows
 // spread over the four lane quadrants and each pair of softmax warps owns a
@@ -431,8 +432,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // issues a small tcgen05.mma only every ~66 cycles, so the QK and PV
   // streams run from two lanes and overlap in the tensor pipe.  Per 16
   // tokens two MMAs, P_hi V and P_lo V, or one for a stacked block (P_hi and
-  // P_lo in the same columns, different lanes).  The first MMA of a run starts a
-  // fresh accumulation (the softmax threads have folded the previous run).
+  // P_lo in the same columns, different lanes).  The first MMA of a run
+  // starts a fresh accumulation (the softmax threads have folded the
+  // previous run).
   if (warp == kPvWarp) {
     if (lane == 0 && my_tiles > 0) {
       constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(M, 256, 0, 1);    // A (P, TMEM), B (V) MN-major
