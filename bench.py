@@ -630,6 +630,18 @@ def verify_traffic(tokens: int):
     return t["read_bytes"] * tokens / t["tokens"] + t["write_bytes"]
 
 
+def staging_layout(shapes: dict, align: int = 256):
+    """Byte offsets of named tensors packed into one flat staging buffer, each
+    slot starting on an ``align``-byte boundary (the calls take 16-byte
+    aligned pointers); ``shapes`` maps a name to ``(numel, element_size)``.
+    Returns ``(offsets, total_bytes)``."""
+    offs, off = {}, 0
+    for name, (numel, esize) in shapes.items():
+        offs[name] = off
+        off += -(-numel * esize // align) * align
+    return offs, off
+
+
 def workload_desc(args) -> str:
     """The workload string of `config`, shared by both arms."""
     import synth
@@ -969,10 +981,7 @@ def main():
     if not args.no_e2e:
         steps = range(args.warmup, args.warmup + args.steps)
         proto = wk.step_inputs(args.warmup)
-        offs, off = {}, 0
-        for k, v in proto.items():  # 256-byte aligned slots of one flat buffer
-            offs[k] = off
-            off += -(-v.numel() * v.element_size() // 256) * 256
+        offs, off = staging_layout({k: (v.numel(), v.element_size()) for k, v in proto.items()})
         dev_flat = torch.empty(off, dtype=torch.uint8, device=dev)
 
         def views(flat):

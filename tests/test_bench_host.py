@@ -1,7 +1,7 @@
 """bench.py's host-side pieces on CPU: the algorithmic byte model the
-roofline divides by, the workload string both arms print, and the guard that
+roofline divides by, the workload string both arms print, the guard that
 reports the captured verify traffic only for the kernel code it was captured
-on."""
+on, and the layout of the end-to-end leg's staging buffer."""
 
 import os
 import shutil
@@ -75,3 +75,13 @@ def test_traffic_guard_follows_the_kernel_code(tmp_path, monkeypatch):
 def test_whole_job_time_per_step():
     assert bench.whole_job_us_per_step(40.0, 10, 1) == pytest.approx(4000.0)
     assert bench.whole_job_us_per_step(40.0, 10, 4) == pytest.approx(1000.0)
+
+
+def test_staging_layout_slots_are_aligned_and_disjoint():
+    shapes = {"q": (3 * 16 * 256, 2), "len": (1, 4), "k": (4 * 2 * 256, 2), "n": (3, 4)}
+    offs, total = bench.staging_layout(shapes)
+    spans = sorted((offs[k], offs[k] + n * e) for k, (n, e) in shapes.items())
+    assert all(o % 256 == 0 for o in offs.values())
+    assert all(a_end <= b_start for (_, a_end), (b_start, _) in zip(spans, spans[1:]))
+    assert spans[-1][1] <= total < spans[-1][1] + 256
+    assert total == sum(-(-n * e // 256) * 256 for n, e in shapes.values())
