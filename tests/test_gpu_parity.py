@@ -114,8 +114,9 @@ def test_custom_softmax_scale():
 # ---------------------------------------------------------------- verify
 @pytest.mark.parametrize("num_q,G,D,P", [(4, 4, 64, 16), (1, 8, 256, 64), (2, 8, 256, 64), (4, 8, 256, 64),
                                          (6, 8, 256, 64), (8, 8, 256, 64), (3, 5, 64, 32), (4, 8, 256, 16),
-                                         # tcgen05 path: 15 rows (odd G), 16 rows, the 64-row maximum
-                                         (3, 5, 256, 32), (4, 4, 256, 128), (4, 16, 256, 256),
+                                         # tcgen05 path: 15 rows (odd G), 16 rows, the 64-row maximum,
+                                         # 33 rows (the first block without spare lanes for P_lo)
+                                         (3, 5, 256, 32), (4, 4, 256, 128), (4, 16, 256, 256), (3, 11, 256, 64),
                                          # tcgen05 with M = 128: gamma = 8 (72 rows), 65 and 128 rows
                                          (9, 8, 256, 64), (5, 13, 256, 64), (8, 16, 256, 32)])
 def test_verify_ragged(num_q, G, D, P):
